@@ -1,0 +1,569 @@
+"""Plain float64 CPU oracle for one blocked-Shampoo optimizer step.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+cpu_baseline / reference leg of ``bench.py`` may import or run this module.
+It shares no code with the CUDA path (no kernels, headers, tables or
+helpers) and imports nothing from it.  It is slow on purpose: every step is
+written the way the pages state it, with NumPy float64 matmuls / ``eigh`` as
+the only library primitives.
+
+Sources (cited by short name below):
+
+[DASH]        "DASH: Faster Shampoo via Batched Block Preconditioning and
+              Efficient Inverse-Root Solvers" (Modoranu, Zmushko, Schultheis,
+              Safaryan, Alistarh; arXiv 2602.02016v2), section summary.
+[DistShampoo] "A Distributed Data-Parallel PyTorch Implementation of the
+              Distributed Shampoo Optimizer for Training Neural Networks
+              At-Scale" (Shi et al.), abstract.
+[3D-Shampoo]  "3D-Shampoo optimizer" README ("Hyperparameters", "Tests").
+[Notes]       "Shampoo" notes (speedrun/shampoo): "The guarantee", the
+              one-sided bounds, "the Kronecker bound", "Roots on idle CPUs",
+              "Spreading the preconditioners", "Grafting corrects ...".
+
+Readings taken where the pages are silent or ambiguous (each one is also a
+row of the readings table in the design notes):
+
+R1  Block order inside a bucket: layers in input order; inside a layer all
+    left factors (blocks row-major) before all right factors; buckets in order
+    of first appearance.  Reproduces the listing order of [DASH] §4.
+R2  Statistics: L <- beta2*L + alpha*G G^T with alpha = 1 by default (the
+    "exponential moving average" of [DASH] §2 is alpha = 1 - beta2).
+R3  Exact root: eigenvalues of L clamped at 0, then eps added once
+    ([DASH] B.1 corrected spectrum).
+R4  Newton-DB is the inverse-free coupled Newton-Schulz / Denman-Beavers
+    form (3 matmuls per iteration, the first iteration closed-form).
+    "iters" counts iterations per call; the second call starts from the
+    first call's Y with Z = I and no re-scaling.
+R5  Coupled Newton (Guo-Higham): M0 = A/s, X0 = I, T = ((p+1)I - M)/p,
+    X <- X T, M <- T^p M.
+R6  Chebyshev: x^{-1/p} fitted at the degree+1 first-kind Chebyshev nodes of
+    [eps, 1+eps]; S = 2 L/s - I with L undamped; result s^{-1/p} p(S).
+R7  Multi-power-iteration: V <- normalise(A V) `iters` times, then the
+    largest Rayleigh quotient v^T A v; start vectors are an input.
+R8  Grafting is layerwise by default; Adam bias-corrected with eps_g; decoupled
+    weight decay W <- W - lr*rho*D - lr*wd*W; rho = 0 when ||D|| = 0.
+
+Parity unpinned: the power-iteration iteration count (R7: no page fixes it),
+the step-count example of [DASH] §3 (Frobenius scaling 5 -> 15 steps).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "BLOCK_FIELDS", "split_dim", "plan_blocks", "stack_gradients", "unstack_directions",
+    "update_stats", "spd_power", "inv_root_exact",
+    "frobenius_scale", "power_iteration_scale",
+    "ndb_matrix", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
+    "cn_matrix", "cn_inv_root", "cn_scalar", "cn_inv_root_replay",
+    "cheb_coefficients", "clenshaw_scalar", "cheb_matrix", "cheb_inv_root", "cheb_inv_root_replay",
+    "inv_root", "precondition", "graft_update", "ShampooState", "shampoo_step",
+    "rel_fro",
+]
+
+# --------------------------------------------------------------------------
+# O1  Block partitioning and stacking
+#     [3D-Shampoo] Hyperparameters (block_size: split dimensions larger than
+#     this; 0 = never split); [DASH] §1 (B x B blocking) and §4 Blocking
+#     Strategy (same-shape blocks stacked into 3D tensors).
+# --------------------------------------------------------------------------
+
+BLOCK_FIELDS = ("layer", "block_row", "block_col", "row0", "col0", "rows", "cols",
+                "g_bucket", "g_index", "l_bucket", "l_index", "r_bucket", "r_index")
+
+
+def split_dim(d: int, block_size: int) -> list[int]:
+    """Sizes of the blocks one dimension is cut into.
+
+    A dimension larger than the block size becomes floor(d/B) blocks of B and
+    one remainder block of d mod B (when nonzero); a dimension <= B, or
+    B = 0, stays whole ([3D-Shampoo] Hyperparameters; [DASH] §4: V = 32000 at
+    B = 1024 gives 31 full rows of blocks and one of 256).
+    """
+    if d <= 0:
+        raise ValueError("dimension must be positive")
+    if block_size <= 0 or d <= block_size:
+        return [d]
+    sizes = [block_size] * (d // block_size)
+    if d % block_size:
+        sizes.append(d % block_size)
+    return sizes
+
+
+def plan_blocks(shapes, block_size: int) -> dict:
+    """Partition every layer into blocks and assign them to stacks.
+
+    Returns int32 tables:
+      blocks    (n_blocks, 13) with the columns of ``BLOCK_FIELDS``;
+      g_buckets (n_g, 3)  rows, cols, count of each gradient-block stack;
+      f_buckets (n_f, 2)  n, count of each preconditioner-factor stack.
+    Gradient blocks are bucketed by (rows, cols), factors by n ([DASH] §4);
+    the order inside buckets is reading R1.
+    """
+    blocks = []
+    g_key_to_id: dict = {}
+    g_counts: list = []
+    f_key_to_id: dict = {}
+    f_counts: list = []
+
+    def f_slot(n):
+        if n not in f_key_to_id:
+            f_key_to_id[n] = len(f_counts)
+            f_counts.append([n, 0])
+        b = f_key_to_id[n]
+        idx = f_counts[b][1]
+        f_counts[b][1] += 1
+        return b, idx
+
+    for li, (m, n) in enumerate(shapes):
+        rs = split_dim(int(m), block_size)
+        cs = split_dim(int(n), block_size)
+        layer_blocks = []
+        row0 = 0
+        for br, r in enumerate(rs):
+            col0 = 0
+            for bc, c in enumerate(cs):
+                key = (r, c)
+                if key not in g_key_to_id:
+                    g_key_to_id[key] = len(g_counts)
+                    g_counts.append([r, c, 0])
+                gb = g_key_to_id[key]
+                gi = g_counts[gb][2]
+                g_counts[gb][2] += 1
+                layer_blocks.append([li, br, bc, row0, col0, r, c, gb, gi, -1, -1, -1, -1])
+                col0 += c
+            row0 += r
+        for blk in layer_blocks:          # all left factors of the layer, row-major
+            blk[9], blk[10] = f_slot(blk[5])
+        for blk in layer_blocks:          # then all right factors, row-major
+            blk[11], blk[12] = f_slot(blk[6])
+        blocks += layer_blocks
+    return {
+        "blocks": np.asarray(blocks, dtype=np.int32).reshape(-1, len(BLOCK_FIELDS)),
+        "g_buckets": np.asarray(g_counts, dtype=np.int32).reshape(-1, 3),
+        "f_buckets": np.asarray(f_counts, dtype=np.int32).reshape(-1, 2),
+    }
+
+
+def stack_gradients(plan: dict, grads) -> list[np.ndarray]:
+    """Copy every layer's gradient blocks into their (count, rows, cols) stacks."""
+    stacks = [np.zeros((int(c), int(r), int(k)), dtype=np.float64) for (r, k, c) in plan["g_buckets"]]
+    for b in plan["blocks"]:
+        li, _, _, r0, c0, r, c, gb, gi = (int(x) for x in b[:9])
+        stacks[gb][gi] = np.asarray(grads[li], dtype=np.float64)[r0:r0 + r, c0:c0 + c]
+    return stacks
+
+
+def unstack_directions(plan: dict, d_stacks, shapes) -> list[np.ndarray]:
+    """Inverse of ``stack_gradients``: scatter blocks back into layer layout."""
+    out = [np.zeros(s, dtype=np.float64) for s in shapes]
+    for b in plan["blocks"]:
+        li, _, _, r0, c0, r, c, gb, gi = (int(x) for x in b[:9])
+        out[li][r0:r0 + r, c0:c0 + c] = d_stacks[gb][gi]
+    return out
+
+
+# --------------------------------------------------------------------------
+# O2  Statistics update  ([DASH] §2 Preliminaries on Shampoo: moving averages
+#     of G G^T and G^T G; beta2 = 1 gives AdaGrad sums)
+# --------------------------------------------------------------------------
+
+def update_stats(G, L, R, beta2: float, alpha: float = 1.0):
+    """L <- beta2 L + alpha G G^T,  R <- beta2 R + alpha G^T G  (reading R2)."""
+    G = np.asarray(G, dtype=np.float64)
+    L_new = beta2 * np.asarray(L, dtype=np.float64) + alpha * (G @ G.T)
+    R_new = beta2 * np.asarray(R, dtype=np.float64) + alpha * (G.T @ G)
+    return L_new, R_new
+
+
+# --------------------------------------------------------------------------
+# O3  Exact inverse root by symmetric eigendecomposition
+#     ([DASH] §3 EVD; B.1: eps added once, corrected spectrum)
+# --------------------------------------------------------------------------
+
+def spd_power(A, r: float, shift: float = 0.0):
+    """Q diag((max(lam,0) + shift)^r) Q^T for symmetric A."""
+    A = np.asarray(A, dtype=np.float64)
+    A = 0.5 * (A + A.T)
+    w, Q = np.linalg.eigh(A)
+    w = np.clip(w, 0.0, None) + shift
+    return (Q * w ** r) @ Q.T
+
+
+def inv_root_exact(L, eps: float, p: int = 4):
+    """(L + eps I)^{-1/p} with L's eigenvalues clamped at zero (reading R3)."""
+    return spd_power(L, -1.0 / p, shift=eps)
+
+
+# --------------------------------------------------------------------------
+# O4  Scaling  ([DASH] §3 Matrix scaling and Power-Iteration; §1)
+# --------------------------------------------------------------------------
+
+def frobenius_scale(L, eps: float = 0.0) -> float:
+    """||L + eps I||_F, the Frobenius-norm scale of [DASH] §3."""
+    A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
+    return float(np.sqrt(np.sum(A * A)))
+
+
+def power_iteration_scale(L, eps: float, starts, iters: int) -> float:
+    """Multi-power-iteration estimate of lambda_max(L + eps I) ([DASH] §3, §1).
+
+    All start vectors (rows of ``starts``) are iterated in parallel:
+    V <- normalise(A V), ``iters`` times; the estimate is the largest Rayleigh
+    quotient v^T A v over the normalised vectors (reading R7).
+    """
+    A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
+    V = np.asarray(starts, dtype=np.float64).T.copy()
+    V /= np.linalg.norm(V, axis=0, keepdims=True)
+    for _ in range(iters):
+        V = A @ V
+        nrm = np.linalg.norm(V, axis=0, keepdims=True)
+        nrm[nrm == 0] = 1.0
+        V /= nrm
+    rq = np.sum(V * (A @ V), axis=0)
+    return float(np.max(rq))
+
+
+# --------------------------------------------------------------------------
+# O4  Newton-DB  ([DASH] §3 Newton-DB: 3 matmuls per iteration, the first
+#     iteration closed-form, inverse fourth root by chaining two calls)
+# --------------------------------------------------------------------------
+
+def ndb_matrix(Y0, iters: int):
+    """Coupled Newton iteration for (Y0^{1/2}, Y0^{-1/2}) in matrix form.
+
+    Z_0 = I;  T_k = (3I - Z_k Y_k)/2;  Y_{k+1} = Y_k T_k;  Z_{k+1} = T_k Z_k.
+    With Z_0 = I the first iteration needs only Y_0 T_0 (T_0 = (3I - Y_0)/2,
+    Z_1 = T_0), so it costs 1 matmul instead of 3.
+    Returns (Y, Z, number_of_matmuls).
+    """
+    if iters < 1:
+        raise ValueError("iters >= 1")
+    Y0 = np.asarray(Y0, dtype=np.float64)
+    I = np.eye(Y0.shape[0])
+    T = 0.5 * (3.0 * I - Y0)
+    Y = Y0 @ T
+    Z = T
+    mm = 1
+    for _ in range(iters - 1):
+        T = 0.5 * (3.0 * I - Z @ Y)
+        Y, Z = Y @ T, T @ Z
+        mm += 3
+    return Y, Z, mm
+
+
+def ndb_inv_root(L, eps: float, s: float, iters: int):
+    """X ~ (L + eps I)^{-1/4} by two chained Newton-DB calls (reading R4).
+
+    Call 1 on A/s gives Y ~ (A/s)^{1/2}; call 2 on that Y gives
+    Z ~ (A/s)^{-1/4}; X = s^{-1/4} Z.  Returns (X, matmuls).
+    """
+    A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
+    Y1, _, m1 = ndb_matrix(A / s, iters)
+    _, Z2, m2 = ndb_matrix(Y1, iters)
+    return s ** -0.25 * Z2, m1 + m2
+
+
+def ndb_scalar(a, iters: int):
+    """The Newton-DB recurrence on scalars (the eigenvalues of Y0)."""
+    a = np.asarray(a, dtype=np.float64)
+    t = 0.5 * (3.0 - a)
+    y, z = a * t, t
+    for _ in range(iters - 1):
+        t = 0.5 * (3.0 - z * y)
+        y, z = y * t, t * z
+    return y, z
+
+
+def ndb_inv_root_replay(L, eps: float, s: float, iters: int):
+    """Same result as ``ndb_inv_root`` via its eigenvalues.
+
+    Every Newton-DB iterate is a polynomial in A, so it shares A's
+    eigenvectors; running the scalar recurrence on each eigenvalue gives the
+    iteration's exact-arithmetic result at O(n^3) instead of O(iters n^3).
+    """
+    L = np.asarray(L, dtype=np.float64)
+    w, Q = np.linalg.eigh(0.5 * (L + L.T))
+    y1, _ = ndb_scalar((w + eps) / s, iters)
+    _, z2 = ndb_scalar(y1, iters)
+    return (Q * (s ** -0.25 * z2)) @ Q.T
+
+
+# --------------------------------------------------------------------------
+# O4  Coupled Newton  ([Notes] "Roots on idle CPUs": coupled Newton, Guo and
+#     Higham / Iannazzo; [DASH] §1, §5)
+# --------------------------------------------------------------------------
+
+def cn_matrix(M0, iters: int, p: int = 4):
+    """Coupled Newton for M0^{-1/p}: X0 = I, T = ((p+1)I - M)/p, X <- X T,
+    M <- T^p M.  Returns (X, matmuls); T^p by binary powering (2 products
+    for p = 4, so 4 matmuls per iteration)."""
+    M = np.asarray(M0, dtype=np.float64)
+    I = np.eye(M.shape[0])
+    X = I.copy()
+    mm = 0
+    for _ in range(iters):
+        T = ((p + 1) * I - M) / p
+        X = X @ T
+        mm += 1
+        Tp, base, e = None, T, p
+        while e:
+            if e & 1:
+                if Tp is None:
+                    Tp = base
+                else:
+                    Tp = Tp @ base
+                    mm += 1
+            e >>= 1
+            if e:
+                base = base @ base
+                mm += 1
+        M = Tp @ M
+        mm += 1
+    return X, mm
+
+
+def cn_inv_root(L, eps: float, s: float, iters: int, p: int = 4):
+    """X ~ (L + eps I)^{-1/p} by coupled Newton on A/s; X = s^{-1/p} X_k."""
+    A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
+    X, mm = cn_matrix(A / s, iters, p)
+    return s ** (-1.0 / p) * X, mm
+
+
+def cn_scalar(a, iters: int, p: int = 4):
+    a = np.asarray(a, dtype=np.float64)
+    m, x = a.copy(), np.ones_like(a)
+    for _ in range(iters):
+        t = ((p + 1) - m) / p
+        x = x * t
+        m = t ** p * m
+    return x
+
+
+def cn_inv_root_replay(L, eps: float, s: float, iters: int, p: int = 4):
+    L = np.asarray(L, dtype=np.float64)
+    w, Q = np.linalg.eigh(0.5 * (L + L.T))
+    x = cn_scalar((w + eps) / s, iters, p)
+    return (Q * (s ** (-1.0 / p) * x)) @ Q.T
+
+
+# --------------------------------------------------------------------------
+# O4  Chebyshev approximation  ([DASH] A.1 real case, A.2 matrix case and the
+#     optimised Clenshaw recurrence with d-1 matmuls)
+# --------------------------------------------------------------------------
+
+def cheb_coefficients(degree: int, eps: float, p: int = 4):
+    """Coefficients c_0..c_d of x^{-1/p} on [eps, 1+eps] in T_k(t), t in [-1, 1].
+
+    Interpolation at the degree+1 first-kind Chebyshev nodes
+    t_j = cos(pi (j + 1/2)/(d+1)), x_j = eps + (t_j + 1)/2 (reading R6):
+    c_k = 2/(d+1) sum_j f(x_j) T_k(t_j), with c_0 halved so the series is
+    sum_k c_k T_k(t).
+    """
+    N = degree + 1
+    j = np.arange(N, dtype=np.float64)
+    theta = math.pi * (j + 0.5) / N
+    x = eps + (np.cos(theta) + 1.0) / 2.0
+    f = x ** (-1.0 / p)
+    c = np.empty(N)
+    for k in range(N):
+        c[k] = 2.0 / N * np.sum(f * np.cos(k * theta))
+    c[0] *= 0.5
+    return c
+
+
+def clenshaw_scalar(c, t):
+    """sum_k c_k T_k(t) by Clenshaw's backward recurrence ([DASH] A.1)."""
+    t = np.asarray(t, dtype=np.float64)
+    b1 = np.zeros_like(t)
+    b2 = np.zeros_like(t)
+    for k in range(len(c) - 1, 0, -1):
+        b1, b2 = c[k] + 2.0 * t * b1 - b2, b1
+    return c[0] + t * b1 - b2
+
+
+def cheb_matrix(S, c):
+    """sum_k c_k T_k(S) by the optimised matrix Clenshaw recurrence ([DASH] A.2).
+
+    B_d = c_d I, B_{d-1} = c_{d-1} I + 2 c_d S, B_k = c_k I + 2 S B_{k+1} - B_{k+2}
+    for k = d-2 .. 1, result c_0 I + S B_1 - B_2: d-1 matmuls in all.
+    Returns (P, matmuls).
+    """
+    S = np.asarray(S, dtype=np.float64)
+    I = np.eye(S.shape[0])
+    d = len(c) - 1
+    if d == 0:
+        return c[0] * I, 0
+    if d == 1:
+        return c[0] * I + c[1] * S, 0
+    b2 = c[d] * I                       # B_{k+2}
+    b1 = c[d - 1] * I + 2.0 * c[d] * S  # B_{k+1}
+    mm = 0
+    for k in range(d - 2, 0, -1):
+        b1, b2 = c[k] * I + 2.0 * (S @ b1) - b2, b1
+        mm += 1
+    P = c[0] * I + S @ b1 - b2
+    return P, mm + 1
+
+
+def cheb_inv_root(L, eps: float, s: float, degree: int, p: int = 4):
+    """X = s^{-1/p} sum_k c_k T_k(2 L/s - I)  ~  (L + s eps I)^{-1/p}."""
+    L = np.asarray(L, dtype=np.float64)
+    S = 2.0 * L / s - np.eye(L.shape[0])
+    P, mm = cheb_matrix(S, cheb_coefficients(degree, eps, p))
+    return s ** (-1.0 / p) * P, mm
+
+
+def cheb_inv_root_replay(L, eps: float, s: float, degree: int, p: int = 4):
+    L = np.asarray(L, dtype=np.float64)
+    w, Q = np.linalg.eigh(0.5 * (L + L.T))
+    x = clenshaw_scalar(cheb_coefficients(degree, eps, p), 2.0 * w / s - 1.0)
+    return (Q * (s ** (-1.0 / p) * x)) @ Q.T
+
+
+def inv_root(L, eps: float, method: str, iters: int, scale: float, p: int = 4, replay: bool = True):
+    """Dispatch to the method (eigenvalue replay when ``replay``)."""
+    if method == "ndb":
+        return ndb_inv_root_replay(L, eps, scale, iters) if replay else ndb_inv_root(L, eps, scale, iters)[0]
+    if method == "cn":
+        return cn_inv_root_replay(L, eps, scale, iters, p) if replay else cn_inv_root(L, eps, scale, iters, p)[0]
+    if method == "cheb":
+        return cheb_inv_root_replay(L, eps, scale, iters, p) if replay else cheb_inv_root(L, eps, scale, iters, p)[0]
+    if method == "evd":
+        return inv_root_exact(L, eps, p)
+    raise ValueError(method)
+
+
+# --------------------------------------------------------------------------
+# O5  Search direction  ([DASH] §2: two-sided preconditioning)
+# --------------------------------------------------------------------------
+
+def precondition(XL, G, XR):
+    """D = L^{-1/4} G R^{-1/4} for one block."""
+    return np.asarray(XL, np.float64) @ np.asarray(G, np.float64) @ np.asarray(XR, np.float64)
+
+
+# --------------------------------------------------------------------------
+# O6  Grafting and parameter update  ([DASH] §2 Adam grafting;
+#     [3D-Shampoo] Hyperparameters graft_type / weight_decay; [Notes]
+#     "Roots on idle CPUs" and "Spreading the preconditioners": grafting
+#     sets each layer's step length)
+# --------------------------------------------------------------------------
+
+def graft_update(W, G, D, m, v, kind: str, lr: float, beta1: float, beta2: float,
+                 eps: float, wd: float, step: int, groups=None):
+    """One grafted update of one layer (reading R8).
+
+    kind: "none" | "sgd" | "adagrad" | "adam".  The graft direction is
+    SGD: G;  AdaGrad: G / (sqrt(v) + eps) with v <- v + G^2;
+    Adam: m_hat / (sqrt(v_hat) + eps) with bias-corrected moments.
+    rho = ||graft||_F / ||D||_F over the layer (or over each entry of
+    ``groups``, a list of index tuples for blockwise grafting), and
+    W <- W - lr rho D - lr wd W.  Returns (W, m, v, rho_list).
+    """
+    W = np.asarray(W, np.float64).copy()
+    G = np.asarray(G, np.float64)
+    D = np.asarray(D, np.float64)
+    m = None if m is None else np.asarray(m, np.float64).copy()
+    v = None if v is None else np.asarray(v, np.float64).copy()
+    if kind == "none":
+        graft = None
+    elif kind == "sgd":
+        graft = G
+    elif kind == "adagrad":
+        v = v + G * G
+        graft = G / (np.sqrt(v) + eps)
+    elif kind == "adam":
+        m = beta1 * m + (1.0 - beta1) * G
+        v = beta2 * v + (1.0 - beta2) * G * G
+        mhat = m / (1.0 - beta1 ** step)
+        vhat = v / (1.0 - beta2 ** step)
+        graft = mhat / (np.sqrt(vhat) + eps)
+    else:
+        raise ValueError(kind)
+    if groups is None:
+        groups = [(slice(None), slice(None))]
+    rhos = []
+    upd = np.zeros_like(W)
+    for sl in groups:
+        if graft is None:
+            rho = 1.0
+        else:
+            dn = math.sqrt(float(np.sum(D[sl] ** 2)))
+            gn = math.sqrt(float(np.sum(graft[sl] ** 2)))
+            rho = gn / dn if dn > 0 else 0.0
+        upd[sl] = rho * D[sl]
+        rhos.append(rho)
+    W = W - lr * upd - lr * wd * W
+    return W, m, v, rhos
+
+
+# --------------------------------------------------------------------------
+# Whole step (composition of O1..O6)
+# --------------------------------------------------------------------------
+
+class ShampooState:
+    """Optimizer state of the oracle: factor stacks and graft moments."""
+
+    def __init__(self, shapes, block_size: int, graft: str):
+        self.shapes = [tuple(int(x) for x in s) for s in shapes]
+        self.plan = plan_blocks(self.shapes, block_size)
+        self.factors = [np.zeros((int(c), int(n), int(n))) for (n, c) in self.plan["f_buckets"]]
+        need = graft in ("adam", "adagrad")
+        self.m = [np.zeros(s) for s in self.shapes] if graft == "adam" else [None] * len(self.shapes)
+        self.v = [np.zeros(s) for s in self.shapes] if need else [None] * len(self.shapes)
+        self.step = 0
+
+
+def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, eps: float,
+                 method: str, iters: int, scaling: str, graft: str, lr: float,
+                 beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
+                 wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
+                 replay: bool = True):
+    """One optimizer step over all layers; returns the new weights.
+
+    ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
+    (bucket, index), so a caller can replay with another scale.
+    """
+    plan = state.plan
+    state.step += 1
+    g_st = stack_gradients(plan, grads)
+    for b in plan["blocks"]:
+        gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
+        state.factors[lb][lix], state.factors[rb][rix] = update_stats(
+            g_st[gb][gi], state.factors[lb][lix], state.factors[rb][rix], beta2, alpha)
+    roots = [np.empty_like(f) for f in state.factors]
+    for fb, stack in enumerate(state.factors):
+        for i in range(stack.shape[0]):
+            Lf = stack[i]
+            if method == "evd":
+                s = 1.0
+            elif scaling == "frobenius":
+                s = frobenius_scale(Lf, 0.0 if method == "cheb" else eps)
+            else:
+                s = power_iteration_scale(Lf, 0.0 if method == "cheb" else eps, pi_starts, pi_iters)
+            if scales_out is not None:
+                scales_out[(fb, i)] = s
+            roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay)
+    d_st = [np.empty_like(g) for g in g_st]
+    for b in plan["blocks"]:
+        gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
+        d_st[gb][gi] = precondition(roots[lb][lix], g_st[gb][gi], roots[rb][rix])
+    D = unstack_directions(plan, d_st, state.shapes)
+    newW = []
+    for li in range(len(state.shapes)):
+        w, m, v, _ = graft_update(W[li], grads[li], D[li], state.m[li], state.v[li], graft, lr,
+                                  beta1, graft_beta2, graft_eps, wd, state.step)
+        state.m[li], state.v[li] = m, v
+        newW.append(w)
+    return newW
+
+
+def rel_fro(x, ref) -> float:
+    """||x - ref||_F / ||ref||_F."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = float(np.linalg.norm(ref))
+    return float(np.linalg.norm(x - ref)) / (den if den > 0 else 1.0)

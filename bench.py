@@ -1,0 +1,417 @@
+"""Benchmark: one blocked-Shampoo optimizer step on B200 (blocks/s, ms/step).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config transformer]
+                [--dtype fp32] [--impl ours|reference]
+
+A step is the whole hot path on one batch of synthetic gradients: gather the
+gradient blocks into stacks, update the statistics, compute every inverse
+fourth root (Newton-DB after power-iteration scaling), precondition, graft
+onto Adam and update the weights.  Inputs are seeded synthetic data already
+resident in HBM; they are larger than L2 (no flush needed).  Rank 0 prints
+one JSON line.  Under torchrun each rank runs its own independent copy of the
+workload (weak scaling, no collective on the data path).
+
+`--impl reference` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (the reference arm); only rank 0 runs.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+# ---------------------------------------------------------------- workloads --
+
+CONFIGS = {
+    # 8 transformer layers, d = 1024, FFN 4096, blocked at 1024: 96 blocks.
+    "transformer": dict(kind="transformer", workload="transformer_8x1024_ffn4096_b1024", shapes="transformer", block_size=1024,
+                        beta2=0.999, alpha=1.0, eps=1e-6, method="ndb", iters=20, scaling="power",
+                        graft="adam", lr=1e-3, weight_decay=0.0),
+    # 256 blocks of 128 x 128 (each block its own layer).
+    "lowrank_stack": dict(kind="lowrank_stack", workload="stack_256x128x128", shapes=[(128, 128)] * 256, block_size=128,
+                          beta2=0.999, alpha=1.0, eps=1e-6, method="ndb", iters=15, scaling="frobenius",
+                          graft="adam", lr=1e-3, weight_decay=0.0),
+    # 32 blocks of 2048 x 2048.
+    "large_blocks": dict(kind="large_blocks", workload="stack_32x2048x2048", shapes=[(2048, 2048)] * 32, block_size=2048,
+                         beta2=0.999, alpha=1.0, eps=1e-6, method="ndb", iters=20, scaling="frobenius",
+                         graft="adam", lr=1e-3, weight_decay=0.01),
+    # one 256 x 256 weight in 16 blocks of 64 x 64
+    "tiny_dense": dict(kind="tiny_dense", workload="dense_256x256_b64", shapes=[(256, 256)], block_size=64, beta2=1.0, alpha=1.0,
+                       eps=1e-6, method="ndb", iters=20, scaling="frobenius", graft="sgd", lr=0.1,
+                       weight_decay=0.0),
+}
+
+
+def shapes_of(cfg):
+    from matrix_roots_b200 import workloads as W
+    return W.transformer_shapes() if cfg["shapes"] == "transformer" else list(cfg["shapes"])
+
+
+def make_grads(shapes, seed, kind="transformer"):
+    """One gradient per layer with the workload's value distribution."""
+    from matrix_roots_b200 import workloads as W
+    if kind == "lowrank_stack":
+        g = W.lowrank_stack_grads(steps=1, blocks=len(shapes), n=shapes[0][0], seed=seed)[0]
+        return [g[i] for i in range(len(shapes))]
+    if kind == "large_blocks":
+        g = W.large_block_grads(steps=1, blocks=len(shapes), n=shapes[0][0], seed=seed)[0]
+        return [g[i] for i in range(len(shapes))]
+    if kind == "tiny_dense":
+        return [W.tiny_dense_grads(steps=1, rows=m, cols=n, seed=seed)[0] for (m, n) in shapes]
+    return W.transformer_grads(shapes, seed=seed)
+
+
+def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters):
+    """Algorithmic FLOPs of one shampoo_inv_root call (2 n^3 per matmul)."""
+    if method == "ndb":
+        mm = 2 * (3 * iters - 3) if iters >= 2 else 2
+    elif method == "cn":
+        mm = 4 * iters - 4 if iters >= 2 else 0
+    else:
+        mm = max(iters - 1, 0)
+    f = mm * 2.0 * n ** 3
+    if scaling == "power":
+        f += (pi_iters + 1) * 2.0 * n * n * pi_vectors
+    return f * count
+
+
+# ------------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- distributed --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local):
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks ----
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sust": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------- cpu baseline ----
+
+def cpu_threads():
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    blas = None
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = max((i.get("num_threads", 0) for i in info), default=None)
+    except Exception:
+        pass
+    return cores, blas
+
+
+def oracle_blocks_per_s(cfg, shapes, sample_blocks, seed=0):
+    """Times the oracle's step on `sample_blocks` gradient blocks of the workload."""
+    import oracle as O
+    from matrix_roots_b200 import workloads as W
+    B = cfg["block_size"]
+    sub = []
+    for (m, n) in shapes:
+        sub.append((min(m, B), min(n, B)))
+        if len(sub) >= sample_blocks:
+            break
+    grads = make_grads(sub, seed, kind=cfg["kind"])
+    st = O.ShampooState(sub, B, cfg["graft"])
+    Wt = [np.zeros(s) for s in sub]
+    starts = None
+    if cfg["scaling"] == "power":
+        starts = W.power_iteration_starts(min(B, max(max(s) for s in sub)), 16)
+    t0 = time.perf_counter()
+    O.shampoo_step(st, Wt, grads, beta2=cfg["beta2"], alpha=cfg["alpha"], eps=cfg["eps"], method=cfg["method"],
+                   iters=cfg["iters"], scaling=cfg["scaling"], graft=cfg["graft"], lr=cfg["lr"],
+                   wd=cfg["weight_decay"], pi_starts=starts, pi_iters=10)
+    dt = time.perf_counter() - t0
+    nblocks = len(O.plan_blocks(sub, B)["blocks"])
+    return nblocks / dt, dt, nblocks
+
+
+# ------------------------------------------------------------------ arms -----
+
+def run_reference(args, cfg):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    shapes = shapes_of(cfg)
+    cores, blas = cpu_threads()
+    for _ in range(args.warmup):
+        oracle_blocks_per_s(cfg, shapes, 1)
+    times, nb = [], 0
+    for _ in range(args.steps):
+        _, dt, nb = oracle_blocks_per_s(cfg, shapes, 1)
+        times.append(dt)
+    ms = 1000 * statistics.median(times)
+    value = nb / (ms / 1000)
+    sample = f"{nb} gradient block(s) of {cfg['workload']} per step (oracle float64 step: stats, eigen-replayed " \
+             f"{cfg['method']} roots, direction, graft)"
+    out = {"metric": "shampoo optimizer step throughput", "value": value, "unit": "blocks/s", "impl": "reference",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": cfg["workload"], "method": cfg["method"], "iters": cfg["iters"]},
+           "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": blas or cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args, cfg):
+    import torch
+    from matrix_roots_b200 import binding as B
+    from matrix_roots_b200 import build
+    from matrix_roots_b200.optimizer import BlockedShampoo, ShampooConfig
+
+    world, rank, local = dist_env()
+    build.build()
+    init_dist(world, local)
+    dev = torch.device("cuda", local)
+    shapes = shapes_of(cfg)
+    scfg = ShampooConfig(block_size=cfg["block_size"], beta2=cfg["beta2"], alpha=cfg["alpha"], eps=cfg["eps"],
+                         method=cfg["method"], iters=cfg["iters"], dtype=args.dtype, stats_dtype=args.dtype,
+                         precond_dtype=args.dtype, scaling=cfg["scaling"], graft=cfg["graft"], lr=cfg["lr"],
+                         weight_decay=cfg["weight_decay"])
+    opt = BlockedShampoo(shapes, scfg, dev)
+    grads_np = make_grads(shapes, seed=rank, kind=args.config)
+    G = [torch.from_numpy(g).to(dev) for g in grads_np]
+    W = [torch.zeros(s, dtype=torch.float32, device=dev) for s in shapes]
+    stream = torch.cuda.current_stream(dev)
+    n_blocks = opt.plan.n_blocks
+
+    # root timing hooks: events around every inv_root call of the timed steps
+    root_events = []
+
+    def step(timed):
+        c = scfg
+        ws = opt.workspace
+        opt.t += 1
+        B.stack_blocks(opt.plan, G, opt.g_stacks)
+        B.update_stats(opt.plan, opt.g_stacks, opt.factors, c.beta2, c.alpha, c.stats_dtype, ws)
+        for fb, (n, _) in enumerate(opt.tables["f_buckets"]):
+            if timed:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            B.inv_root(opt.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
+                       opt.pi_starts.get(int(n)), opt.roots[fb], opt.scales[fb], opt.status[fb], ws)
+            if timed:
+                e1.record(stream)
+                root_events.append((e0, e1, int(n), int(opt.tables["f_buckets"][fb][1])))
+        B.precondition(opt.plan, opt.roots, opt.g_stacks, opt.d_stacks, opt.dnorm2, c.precond_dtype, ws)
+        B.graft_step(opt.plan, W, G, opt.d_stacks, opt.dnorm2, opt.m, opt.v, c.graft, c.lr, c.beta1,
+                     c.graft_beta2, c.graft_eps, c.weight_decay, opt.t, c.graft_per_block, ws)
+
+    for _ in range(args.warmup):
+        step(False)
+    barrier(world)
+    assert B.device_error() == 0, "a kernel reported a barrier timeout during warm-up"
+    for s in opt.status:
+        assert int(s.abs().sum()) == 0, "non-finite root during warm-up"
+
+    l0 = B.launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        barrier(world)
+    launches = B.launch_count() - l0
+    ms_total = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms_total, world)
+    ms_step = ms_max / args.steps
+    value = world * n_blocks * args.steps / (ms_max / 1000.0)
+
+    # roofline of the dominant kernel (the tcgen05 GEMM engine inside inv_root)
+    root_ms = sum(a.elapsed_time(b) for a, b, _, _ in root_events) / args.steps
+    flops = sum(root_flops(n, c, scfg.method, scfg.iters, scfg.scaling, scfg.pi_vectors, scfg.pi_iters)
+                for _, _, n, c in root_events) / args.steps
+    peaks = load_peaks()
+    tf32_sust = 0.5 * peaks["bf16_sust"]  # nominal dense TF32 / BF16 = 1/2
+    passes = {"fp32": 3.0, "tf32": 1.0, "fp16": 0.5, "bf16": 0.5}[args.dtype]
+    peak = tf32_sust / passes
+    achieved = flops / (root_ms / 1000.0) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None,
+                "kernel": "gemm_kernel (all launches inside shampoo_inv_root)",
+                "peak_note": f"{peaks['source']} sustained bf16 x 0.5 (TF32) / {passes:g} MMA passes per "
+                             f"algorithmic flop ({args.dtype})",
+                "root_ms_per_step": root_ms, "root_tflop_per_step": flops / 1e12}
+
+    # end to end through the public API with host-resident gradients and weights
+    e2e = None
+    if not args.no_e2e:
+        G_host = [g.cpu().pin_memory() for g in G]
+        W_host = [torch.empty(s, dtype=torch.float32).pin_memory() for s in shapes]
+        h2d = sum(g.numel() * 4 for g in G_host)
+        d2h = sum(w.numel() * 4 for w in W_host)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(args.steps):
+            for gd, gh in zip(G, G_host):
+                gd.copy_(gh, non_blocking=True)
+            step(False)
+            for wh, wd in zip(W_host, W):
+                wh.copy_(wd, non_blocking=True)
+        e1.record(stream)
+        barrier(world)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": world * n_blocks * args.steps / (e_ms / 1000.0), "unit": "blocks/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}
+
+    out = None
+    if rank == 0:
+        out = {"metric": "shampoo optimizer step throughput", "value": value, "unit": "blocks/s",
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": {"fp32": "f32 (3xTF32 tensor-core split)", "tf32": "tf32", "fp16": "f16",
+                         "bf16": "bf16"}[args.dtype],
+               "data": "synthetic",
+               "config": {"workload": cfg["workload"], "blocks_per_gpu": n_blocks, "factors_per_gpu":
+                          int(sum(int(c) for _, c in opt.tables["f_buckets"])), "method": cfg["method"],
+                          "iters": cfg["iters"], "scaling": cfg["scaling"], "graft": cfg["graft"],
+                          "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+               "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
+               "clocks": clocks.summary()}
+        if world == 1 and not args.no_cpu:
+            cores, blas = cpu_threads()
+            rate, dt, nb = oracle_blocks_per_s(cfg, shapes, args.cpu_blocks)
+            out["cpu_baseline"] = {"value": rate, "unit": "blocks/s", "cores": blas or cores, "kind": "oracle",
+                                   "sample": f"{nb} of the {n_blocks} gradient blocks, one oracle step "
+                                             f"({dt:.1f} s)"}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="transformer", choices=sorted(CONFIGS))
+    ap.add_argument("--dtype", default="fp32", choices=["fp32", "tf32", "fp16", "bf16"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-blocks", type=int, default=4)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

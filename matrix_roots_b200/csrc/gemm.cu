@@ -1,0 +1,413 @@
+// Batched tcgen05 GEMM with fused epilogues, the contraction engine behind
+// the statistics update, every inverse-root iteration and the two-sided
+// preconditioning ("DASH: Faster Shampoo via Batched Block Preconditioning
+// and Efficient Inverse-Root Solvers", §4: same-shape blocks stacked into 3D
+// tensors and processed by batched matmuls).
+//
+// One CTA computes a 128 x BN tile of one matrix of the stack:
+//   warp 5      TMA producer: 128B-swizzled operand tiles into a STAGES-deep
+//               shared-memory ring (mbarrier complete_tx)
+//   warp 4      TMEM allocator + single-thread tcgen05.mma issuer; FP32 mode
+//               issues lo*hi + hi*lo + hi*hi (3 x TF32) per K step
+//   warps 0..3  epilogue: tcgen05.ld of the FP32 accumulator, the fused
+//               a*D + b*C + c*I combination, norm / finiteness reductions
+//               and the plane writes the next GEMM reads.
+#include <atomic>
+#include <cstdio>
+#include <mutex>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "internal.h"
+
+namespace shp {
+__device__ int shp_dev_error = 0;
+}  // namespace shp
+
+#define SHP_DEV_ERROR_DEFINED
+#include "ptx.cuh"
+
+namespace shp {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+unsigned long long launch_total() { return g_launches.load(std::memory_order_relaxed); }
+
+cudaError_t read_and_clear_dev_error(int* out) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, shp_dev_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(shp_dev_error, &zero, sizeof(int));
+}
+
+namespace {
+
+template <int KIND>
+struct KindTraits;
+template <>
+struct KindTraits<0> {  // tf32
+  static constexpr int ESZ = 4;
+  static constexpr uint32_t FMT = 2;
+  static constexpr int KINST = 8;
+};
+template <>
+struct KindTraits<1> {  // f16
+  static constexpr int ESZ = 2;
+  static constexpr uint32_t FMT = 0;
+  static constexpr int KINST = 16;
+};
+template <>
+struct KindTraits<2> {  // bf16
+  static constexpr int ESZ = 2;
+  static constexpr uint32_t FMT = 1;
+  static constexpr int KINST = 16;
+};
+
+template <int KIND, int NPASS, int BN>
+struct Cfg {
+  static constexpr int NPL = (NPASS == 3) ? 2 : 1;
+  static constexpr int ESZ = KindTraits<KIND>::ESZ;
+  static constexpr int BKE = 128 / ESZ;  // K elements per stage (one 128-byte swizzle row)
+  static constexpr int A_TILE = 128 * 128;
+  static constexpr int B_TILE = BN * 128;
+  static constexpr int STAGE_BYTES = NPL * (A_TILE + B_TILE);
+  static constexpr int SMEM_BUDGET = 227 * 1024 - 2048;
+  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(STAGES >= 2, "tile does not fit shared memory");
+};
+
+__device__ __forceinline__ void store_h16(void* base, long long off, float v, int bf) {
+  if (bf)
+    reinterpret_cast<__nv_bfloat16*>(base)[off] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<__half*>(base)[off] = __float2half_rn(v);
+}
+
+__device__ __forceinline__ void write_out(const EpiOut& o, long long off, float r) {
+  if (o.lo) {
+    const float hi = tf32_round(r);
+    o.f32[off] = hi;
+    o.lo[off] = r - hi;
+  } else if (o.f32) {
+    o.f32[off] = r;
+  }
+  if (o.h16) store_h16(o.h16, off, r, o.h16_bf);
+}
+
+template <int KIND, int NPASS, int BN>
+__global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<KIND, NPASS, BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int z = blockIdx.z;
+  const int grp = z / p.batch;
+  const int b = z - grp * p.batch;
+  const GroupDev& g = p.g[grp];
+  const int m0 = blockIdx.y * 128;
+  const int n0 = blockIdx.x * BN;
+  if (m0 >= g.M || n0 >= g.N) return;  // uniform for the whole CTA
+  // once any CTA has given up on a barrier, later CTAs skip their tile
+  // instead of each waiting out its own time limit
+  if (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) return;
+  const int nk = (g.K + C::BKE - 1) / C::BKE;
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accum_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 5) {
+    if (lane == 0) {
+      const CUtensorMap* mA0 = &p.tmA[grp][0];
+      const CUtensorMap* mA1 = &p.tmA[grp][1];
+      const CUtensorMap* mB0 = &p.tmB[grp][0];
+      const CUtensorMap* mB1 = &p.tmB[grp][1];
+      const int ab = g.a_idx ? g.a_idx[b] : b;
+      const int bb = g.b_idx ? g.b_idx[b] : b;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        if (kb >= STAGES && !mbar_wait(empty0 + 8 * s, ((kb / STAGES) - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * s;
+        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+        const int k0 = kb * C::BKE;
+        uint8_t* st = smem + s * C::STAGE_BYTES;
+#pragma unroll
+        for (int pl = 0; pl < C::NPL; ++pl) {
+          const CUtensorMap* ma = pl ? mA1 : mA0;
+          const CUtensorMap* mb = pl ? mB1 : mB0;
+          const uint32_t sa = smem_u32(st + pl * C::A_TILE);
+          const uint32_t sb = smem_u32(st + C::NPL * C::A_TILE + pl * C::B_TILE);
+          if (!g.a_mn) {
+            tma_load_3d(sa, ma, fb, k0, m0, ab);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 128 / C::BKE; ++j) tma_load_3d(sa + j * C::BKE * 128, ma, fb, m0 + j * C::BKE, k0, ab);
+          }
+          if (!g.b_mn) {
+            tma_load_3d(sb, mb, fb, k0, n0, bb);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / C::BKE; ++j) tma_load_3d(sb + j * C::BKE * 128, mb, fb, n0 + j * C::BKE, k0, bb);
+          }
+        }
+      }
+    }
+  } else if (warp == 4) {
+    if (lane == 0) {
+      constexpr uint32_t FMT = KindTraits<KIND>::FMT;
+      const uint32_t idesc = idesc_f32acc(FMT, FMT, g.a_mn, g.b_mn, 128, BN);
+      // byte step of one MMA K-slice inside a stage, per operand major-ness
+      constexpr uint32_t KSTEP_K = KindTraits<KIND>::KINST * C::ESZ;  // 32 bytes
+      constexpr uint32_t KSTEP_MN = KindTraits<KIND>::KINST * 128;     // KINST rows of 128 bytes
+      constexpr uint32_t LBO_MN = C::BKE * 128;                          // one TMA box along M/N
+      const uint32_t a_step = g.a_mn ? KSTEP_MN : KSTEP_K;
+      const uint32_t b_step = g.b_mn ? KSTEP_MN : KSTEP_K;
+      const uint32_t a_lbo = g.a_mn ? LBO_MN : 16u;
+      const uint32_t b_lbo = g.b_mn ? LBO_MN : 16u;
+      // MN-major tf32 tiles use the 32-byte-atom swizzle (4-row atoms, 512 B)
+      constexpr bool MN32 = (KIND == 0);
+      const uint32_t a_lay = (g.a_mn && MN32) ? 1u : 2u;
+      const uint32_t b_lay = (g.b_mn && MN32) ? 1u : 2u;
+      const uint32_t a_sbo = (g.a_mn && MN32) ? 512u : 1024u;
+      const uint32_t b_sbo = (g.b_mn && MN32) ? 512u : 1024u;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        if (!mbar_wait(full0 + 8 * s, (kb / STAGES) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* st = smem + s * C::STAGE_BYTES;
+        const uint32_t sa0 = smem_u32(st);
+        const uint32_t sb0 = smem_u32(st + C::NPL * C::A_TILE);
+#pragma unroll
+        for (int ks = 0; ks < C::BKE / KindTraits<KIND>::KINST; ++ks) {
+          const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
+          const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
+          const uint32_t acc = (kb | ks) ? 1u : 0u;
+          if constexpr (NPASS == 3) {
+            const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
+            mma_tf32(tmem, a_lo, b_hi, idesc, acc);
+            mma_tf32(tmem, a_hi, b_lo, idesc, 1u);
+            mma_tf32(tmem, a_hi, b_hi, idesc, 1u);
+          } else if constexpr (KIND == 0) {
+            mma_tf32(tmem, a_hi, b_hi, idesc, acc);
+          } else {
+            mma_f16(tmem, a_hi, b_hi, idesc, acc);
+          }
+        }
+        tc_commit(empty0 + 8 * s);
+      }
+      tc_commit(accum_bar);  // also on abort, so the epilogue never waits forever
+    }
+  } else {
+    // ---------------- epilogue: warps 0..3, thread <-> accumulator row ----
+    const bool ok = mbar_wait(accum_bar, 0);
+    tc_fence_after();
+    __syncwarp();
+    if (ok && !*abort_flag) {
+      const int row = m0 + warp * 32 + lane;
+      const bool row_ok = row < g.M;
+      const int ob = g.o_idx ? g.o_idx[b] : b;
+      const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+      const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
+      const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
+      const long long crow = (long long)ob * g.C.bs + (long long)row * g.C.ld;
+      const long long orow = (long long)ob * g.O.bs + (long long)row * g.O.ld;
+      const long long xrow = (long long)ob * g.X.bs + (long long)row * g.X.ld;
+      float ss = 0.f;
+      int bad = 0;
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        if (n0 + c0 >= g.N) break;  // uniform across the warp
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+        if (!row_ok) continue;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = n0 + c0 + i;
+          if (col < g.N) {
+            float cval = 0.f;
+            if (need_c) {
+              cval = g.C.f32[crow + col];
+              if (g.C.lo) cval += g.C.lo[crow + col];
+            }
+            const float diag = (row == col) ? 1.f : 0.f;
+            const float r0 = g.alpha * v[i] + g.beta * cval + g.gamma * diag;
+            const float r = r0 * mult;
+            write_out(g.O, orow + col, r);
+            ss += r * r;
+            bad |= !isfinite(r);
+            if (has_x) write_out(g.X, xrow + col, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
+          }
+        }
+      }
+      if (g.sumsq) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) atomicAdd(g.sumsq + ob, ss);
+      }
+      if (g.status && bad) atomicOr(g.status + ob, 1);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+// ---- host side -------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Tensor map over one plane of a stack; box = {bx elements, by rows, 1}.
+// atom32: 128-byte swizzle with 32-byte atoms (MN-major tf32 operands).
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esz, const Planes& P, int bx, int by,
+              bool atom32) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !base) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)P.cols, (cuuint64_t)P.rows, (cuuint64_t)P.count};
+  cuuint64_t strides[2] = {(cuuint64_t)P.ld * esz, (cuuint64_t)P.bs * esz};
+  cuuint32_t box[3] = {(cuuint32_t)bx, (cuuint32_t)by, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int KIND, int NPASS, int BN>
+cudaError_t run(GemmParams& prm, int ngroups, int batch, int maxM, int maxN, cudaStream_t stream) {
+  using C = Cfg<KIND, NPASS, BN>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<KIND, NPASS, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  dim3 grid((maxN + BN - 1) / BN, (maxM + 127) / 128, ngroups * batch);
+  gemm_kernel<KIND, NPASS, BN><<<grid, 192, C::SMEM_BYTES, stream>>>(prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec prec, cudaStream_t stream) {
+  if (ngroups < 1 || ngroups > 2 || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
+  const int kind = (prec == P_FP16) ? 1 : (prec == P_BF16) ? 2 : 0;
+  const int npass = (prec == P_FP32) ? 3 : 1;
+  const int esz = kind ? 2 : 4;
+  const int bke = 128 / esz;
+  const CUtensorMapDataType dt = kind == 0   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  int maxM = 0, maxN = 0, minN = 1 << 30;
+  for (int i = 0; i < ngroups; ++i) {
+    maxM = groups[i].M > maxM ? groups[i].M : maxM;
+    maxN = groups[i].N > maxN ? groups[i].N : maxN;
+    minN = groups[i].N < minN ? groups[i].N : minN;
+  }
+  // Tile width: the widest that still yields a few waves of CTAs.
+  int BN = 256;
+  if (npass == 3) BN = 128;
+  if (maxN <= 64) BN = 64;
+  else if (maxN <= 128) BN = 128;
+
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.ngroups = ngroups;
+  prm.batch = batch;
+  for (int i = 0; i < ngroups; ++i) {
+    const GemmGroup& G = groups[i];
+    if (G.M < 1 || G.N < 1 || G.K < 1) return cudaErrorInvalidValue;
+    GroupDev d = G.epi;
+    d.M = G.M;
+    d.N = G.N;
+    d.K = G.K;
+    d.a_mn = G.a_mn;
+    d.b_mn = G.b_mn;
+    d.a_idx = G.a_idx;
+    d.b_idx = G.b_idx;
+    prm.g[i] = d;
+    for (int pl = 0; pl < npass / 2 + 1 && pl < 2; ++pl) {
+      const void* abase = kind ? G.A->h16 : (pl ? (const void*)G.A->lo : (const void*)G.A->f32);
+      const void* bbase = kind ? G.B->h16 : (pl ? (const void*)G.B->lo : (const void*)G.B->f32);
+      const int abx = bke, aby = G.a_mn ? bke : 128;
+      const int bbx = bke, bby = G.b_mn ? bke : BN;
+      if (!make_map(&prm.tmA[i][pl], abase, dt, esz, *G.A, abx, aby, kind == 0 && G.a_mn))
+        return cudaErrorInvalidValue;
+      if (!make_map(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bbx, bby, kind == 0 && G.b_mn))
+        return cudaErrorInvalidValue;
+    }
+  }
+  if (kind == 0 && npass == 3) {
+    if (BN == 64) return run<0, 3, 64>(prm, ngroups, batch, maxM, maxN, stream);
+    return run<0, 3, 128>(prm, ngroups, batch, maxM, maxN, stream);
+  }
+  if (kind == 0) {
+    if (BN == 64) return run<0, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
+    if (BN == 128) return run<0, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
+    return run<0, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
+  }
+  if (kind == 1) {
+    if (BN == 64) return run<1, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
+    if (BN == 128) return run<1, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
+    return run<1, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
+  }
+  if (BN == 64) return run<2, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
+  if (BN == 128) return run<2, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
+  return run<2, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
+}
+
+}  // namespace shp

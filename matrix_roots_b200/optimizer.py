@@ -1,0 +1,88 @@
+"""One blocked-Shampoo optimizer step as a sequence of the five C-ABI calls.
+
+``BlockedShampoo`` owns the device state (gradient / factor / root /
+direction stacks, graft moments and one shared workspace) and calls, in
+order: shampoo_stack_blocks, shampoo_update_stats, shampoo_inv_root (once
+per factor bucket), shampoo_precondition and shampoo_graft_step.  Every
+arithmetic step runs in the library's CUDA kernels; this module only
+allocates tensors and marshals arguments.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+from . import binding as B
+from . import workloads
+
+
+@dataclass
+class ShampooConfig:
+    block_size: int = 1024
+    beta2: float = 1.0          # statistics decay
+    alpha: float = 1.0          # statistics weight (1 - beta2 for a moving average)
+    eps: float = 1e-6
+    method: str = "ndb"
+    iters: int = 20             # iterations per call, or the Chebyshev degree
+    dtype: str = "fp32"         # root iterations
+    stats_dtype: str = "fp32"
+    precond_dtype: str = "fp32"
+    scaling: str = "frobenius"
+    pi_vectors: int = 16
+    pi_iters: int = 10
+    pi_seed: int = 0
+    graft: str = "sgd"
+    lr: float = 0.1
+    beta1: float = 0.9
+    graft_beta2: float = 0.999
+    graft_eps: float = 1e-8
+    weight_decay: float = 0.0
+    graft_per_block: bool = False
+
+
+class BlockedShampoo:
+    def __init__(self, shapes, cfg: ShampooConfig, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.shapes = [(int(m), int(n)) for m, n in shapes]
+        self.plan = B.Plan(self.shapes, cfg.block_size).bind(self.device)
+        t = self.plan.tables()
+        self.tables = t
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.g_stacks = [torch.empty((int(c), int(r), int(k)), **f32) for r, k, c in t["g_buckets"]]
+        self.d_stacks = [torch.empty_like(g) for g in self.g_stacks]
+        self.factors = [torch.zeros((int(c), int(n), int(n)), **f32) for n, c in t["f_buckets"]]
+        self.roots = [torch.empty_like(f) for f in self.factors]
+        self.scales = [torch.empty(int(c), **f32) for _, c in t["f_buckets"]]
+        self.status = [torch.empty(int(c), dtype=torch.int32, device=self.device) for _, c in t["f_buckets"]]
+        self.dnorm2 = torch.empty(self.plan.n_blocks, **f32)
+        self.m = [torch.zeros(s, **f32) for s in self.shapes] if cfg.graft == "adam" else None
+        self.v = [torch.zeros(s, **f32) for s in self.shapes] if cfg.graft in ("adam", "adagrad") else None
+        self.pi_starts = {}
+        if cfg.scaling == "power":
+            for n, _ in t["f_buckets"]:
+                s = workloads.power_iteration_starts(int(n), cfg.pi_vectors, cfg.pi_seed)
+                self.pi_starts[int(n)] = torch.from_numpy(s).to(self.device)
+        need = max(
+            [B.update_stats_workspace_bytes(self.plan, cfg.stats_dtype),
+             B.precondition_workspace_bytes(self.plan, cfg.precond_dtype),
+             B.graft_step_workspace_bytes(self.plan)]
+            + [B.inv_root_workspace_bytes(int(c), int(n), cfg.method, cfg.dtype, cfg.scaling, cfg.pi_vectors)
+               for n, c in t["f_buckets"]])
+        self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        self.t = 0
+
+    def step(self, W, G, stream=None) -> None:
+        """W <- W - lr * rho * D - lr * wd * W for every layer, in place."""
+        c = self.cfg
+        ws = self.workspace
+        self.t += 1
+        B.stack_blocks(self.plan, G, self.g_stacks, stream)
+        B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
+        for fb, (n, _) in enumerate(self.tables["f_buckets"]):
+            B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
+                       self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
+        B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,
+                       stream)
+        B.graft_step(self.plan, W, G, self.d_stacks, self.dnorm2, self.m, self.v, c.graft, c.lr, c.beta1,
+                     c.graft_beta2, c.graft_eps, c.weight_decay, self.t, c.graft_per_block, ws, stream)

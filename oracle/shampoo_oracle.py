@@ -60,7 +60,7 @@ __all__ = [
     "cn_matrix", "cn_inv_root", "cn_scalar", "cn_inv_root_replay",
     "cheb_coefficients", "clenshaw_scalar", "cheb_matrix", "cheb_inv_root", "cheb_inv_root_replay",
     "inv_root", "precondition", "graft_update", "ShampooState", "shampoo_step",
-    "rel_fro",
+    "rel_fro", "round_mantissa", "truncate_mantissa", "precision_floor",
 ]
 
 # --------------------------------------------------------------------------
@@ -227,43 +227,105 @@ def power_iteration_scale(L, eps: float, starts, iters: int) -> float:
 
 
 # --------------------------------------------------------------------------
+# Arithmetic models.  The matrix-form iterations below run in float64 by
+# default (the oracle).  Given `prec`, the same steps run with float32
+# storage and float32-accumulated products whose operands are first reduced
+# to the named format: "fp32" (none), "tf32" (10 explicit mantissa bits,
+# truncated), "bf16" (7 bits, rounded), "fp16" (IEEE half, rounded).  This models what an arithmetic can
+# reach; tests use it only to derive error bounds ([DASH] A.3 and §5 report
+# that reduced precision changes the result), never as an expected value.
+# --------------------------------------------------------------------------
+
+def round_mantissa(x, bits: int):
+    """Round float32 values to `bits` explicit mantissa bits, ties to even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    drop = 23 - bits
+    lsb = (u >> np.uint64(drop)) & np.uint64(1)
+    u = (u + np.uint64((1 << (drop - 1)) - 1) + lsb) & ~np.uint64((1 << drop) - 1)
+    return u.astype(np.uint32).view(np.float32).reshape(x.shape)
+
+
+def _model(prec):
+    """(matmul, store) of an arithmetic model; prec None = float64."""
+    if prec is None:
+        return (lambda a, b: a @ b), (lambda x: x)
+
+    def f32(x):
+        return np.asarray(x, dtype=np.float32)
+
+    rnd = {"fp32": f32,
+           "tf32": lambda x: truncate_mantissa(x, 10),
+           "bf16": lambda x: round_mantissa(x, 7),
+           "fp16": lambda x: f32(x).astype(np.float16).astype(np.float32)}[prec]
+    return (lambda a, b: rnd(a) @ rnd(b)), f32
+
+
+def truncate_mantissa(x, bits: int):
+    """Keep `bits` explicit mantissa bits of float32 values (round toward 0).
+
+    A TF32 tensor-core pass reads 32-bit operands and ignores their low 13
+    mantissa bits, so the "tf32" model truncates rather than rounds."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    mask = np.uint32((0xFFFFFFFF << (23 - bits)) & 0xFFFFFFFF)
+    return (x.view(np.uint32) & mask).view(np.float32).reshape(x.shape)
+
+
+def precision_floor(L, eps: float, s: float, method: str, iters: int, prec: str, p: int = 4) -> float:
+    """Relative Frobenius error the method reaches in arithmetic model `prec`.
+
+    Runs the matrix-form iteration in the model and compares it with the
+    float64 eigenvalue replay.  Used to derive test tolerances where the
+    input's conditioning puts the stated ones beyond the arithmetic.
+    """
+    fn = {"ndb": ndb_inv_root, "cn": cn_inv_root, "cheb": cheb_inv_root}[method]
+    if method == "ndb":
+        X, _ = fn(L, eps, s, iters, prec)
+    else:
+        X, _ = fn(L, eps, s, iters, p, prec)
+    return rel_fro(X, inv_root(L, eps, method, iters, s, p))
+
+
+# --------------------------------------------------------------------------
 # O4  Newton-DB  ([DASH] §3 Newton-DB: 3 matmuls per iteration, the first
 #     iteration closed-form, inverse fourth root by chaining two calls)
 # --------------------------------------------------------------------------
 
-def ndb_matrix(Y0, iters: int):
+def ndb_matrix(Y0, iters: int, prec=None):
     """Coupled Newton iteration for (Y0^{1/2}, Y0^{-1/2}) in matrix form.
 
     Z_0 = I;  T_k = (3I - Z_k Y_k)/2;  Y_{k+1} = Y_k T_k;  Z_{k+1} = T_k Z_k.
     With Z_0 = I the first iteration needs only Y_0 T_0 (T_0 = (3I - Y_0)/2,
     Z_1 = T_0), so it costs 1 matmul instead of 3.
-    Returns (Y, Z, number_of_matmuls).
+    Returns (Y, Z, number_of_matmuls).  `prec`: arithmetic model (above).
     """
     if iters < 1:
         raise ValueError("iters >= 1")
-    Y0 = np.asarray(Y0, dtype=np.float64)
-    I = np.eye(Y0.shape[0])
-    T = 0.5 * (3.0 * I - Y0)
-    Y = Y0 @ T
+    mul, st = _model(prec)
+    Y0 = st(np.asarray(Y0, dtype=np.float64))
+    I = st(np.eye(Y0.shape[0]))
+    T = st(0.5 * (3.0 * I - Y0))
+    Y = st(mul(Y0, T))
     Z = T
     mm = 1
     for _ in range(iters - 1):
-        T = 0.5 * (3.0 * I - Z @ Y)
-        Y, Z = Y @ T, T @ Z
+        T = st(0.5 * (3.0 * I - st(mul(Z, Y))))
+        Y, Z = st(mul(Y, T)), st(mul(T, Z))
         mm += 3
     return Y, Z, mm
 
 
-def ndb_inv_root(L, eps: float, s: float, iters: int):
+def ndb_inv_root(L, eps: float, s: float, iters: int, prec=None):
     """X ~ (L + eps I)^{-1/4} by two chained Newton-DB calls (reading R4).
 
     Call 1 on A/s gives Y ~ (A/s)^{1/2}; call 2 on that Y gives
     Z ~ (A/s)^{-1/4}; X = s^{-1/4} Z.  Returns (X, matmuls).
     """
+    _, st = _model(prec)
     A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
-    Y1, _, m1 = ndb_matrix(A / s, iters)
-    _, Z2, m2 = ndb_matrix(Y1, iters)
-    return s ** -0.25 * Z2, m1 + m2
+    Y1, _, m1 = ndb_matrix(st(A / s), iters, prec)
+    _, Z2, m2 = ndb_matrix(Y1, iters, prec)
+    return s ** -0.25 * np.asarray(Z2, np.float64), m1 + m2
 
 
 def ndb_scalar(a, iters: int):
@@ -296,17 +358,18 @@ def ndb_inv_root_replay(L, eps: float, s: float, iters: int):
 #     Higham / Iannazzo; [DASH] §1, §5)
 # --------------------------------------------------------------------------
 
-def cn_matrix(M0, iters: int, p: int = 4):
+def cn_matrix(M0, iters: int, p: int = 4, prec=None):
     """Coupled Newton for M0^{-1/p}: X0 = I, T = ((p+1)I - M)/p, X <- X T,
     M <- T^p M.  Returns (X, matmuls); T^p by binary powering (2 products
     for p = 4, so 4 matmuls per iteration)."""
-    M = np.asarray(M0, dtype=np.float64)
-    I = np.eye(M.shape[0])
+    mul, st = _model(prec)
+    M = st(np.asarray(M0, dtype=np.float64))
+    I = st(np.eye(M.shape[0]))
     X = I.copy()
     mm = 0
     for _ in range(iters):
-        T = ((p + 1) * I - M) / p
-        X = X @ T
+        T = st(((p + 1) * I - M) / p)
+        X = st(mul(X, T))
         mm += 1
         Tp, base, e = None, T, p
         while e:
@@ -314,22 +377,23 @@ def cn_matrix(M0, iters: int, p: int = 4):
                 if Tp is None:
                     Tp = base
                 else:
-                    Tp = Tp @ base
+                    Tp = st(mul(Tp, base))
                     mm += 1
             e >>= 1
             if e:
-                base = base @ base
+                base = st(mul(base, base))
                 mm += 1
-        M = Tp @ M
+        M = st(mul(Tp, M))
         mm += 1
     return X, mm
 
 
-def cn_inv_root(L, eps: float, s: float, iters: int, p: int = 4):
+def cn_inv_root(L, eps: float, s: float, iters: int, p: int = 4, prec=None):
     """X ~ (L + eps I)^{-1/p} by coupled Newton on A/s; X = s^{-1/p} X_k."""
+    _, st = _model(prec)
     A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
-    X, mm = cn_matrix(A / s, iters, p)
-    return s ** (-1.0 / p) * X, mm
+    X, mm = cn_matrix(st(A / s), iters, p, prec)
+    return s ** (-1.0 / p) * np.asarray(X, np.float64), mm
 
 
 def cn_scalar(a, iters: int, p: int = 4):
@@ -384,36 +448,38 @@ def clenshaw_scalar(c, t):
     return c[0] + t * b1 - b2
 
 
-def cheb_matrix(S, c):
+def cheb_matrix(S, c, prec=None):
     """sum_k c_k T_k(S) by the optimised matrix Clenshaw recurrence ([DASH] A.2).
 
     B_d = c_d I, B_{d-1} = c_{d-1} I + 2 c_d S, B_k = c_k I + 2 S B_{k+1} - B_{k+2}
     for k = d-2 .. 1, result c_0 I + S B_1 - B_2: d-1 matmuls in all.
     Returns (P, matmuls).
     """
-    S = np.asarray(S, dtype=np.float64)
-    I = np.eye(S.shape[0])
+    mul, st = _model(prec)
+    S = st(np.asarray(S, dtype=np.float64))
+    I = st(np.eye(S.shape[0]))
     d = len(c) - 1
     if d == 0:
         return c[0] * I, 0
     if d == 1:
-        return c[0] * I + c[1] * S, 0
-    b2 = c[d] * I                       # B_{k+2}
-    b1 = c[d - 1] * I + 2.0 * c[d] * S  # B_{k+1}
+        return st(c[0] * I + c[1] * S), 0
+    b2 = st(c[d] * I)                       # B_{k+2}
+    b1 = st(c[d - 1] * I + 2.0 * c[d] * S)  # B_{k+1}
     mm = 0
     for k in range(d - 2, 0, -1):
-        b1, b2 = c[k] * I + 2.0 * (S @ b1) - b2, b1
+        b1, b2 = st(c[k] * I + 2.0 * st(mul(S, b1)) - b2), b1
         mm += 1
-    P = c[0] * I + S @ b1 - b2
+    P = st(c[0] * I + st(mul(S, b1)) - b2)
     return P, mm + 1
 
 
-def cheb_inv_root(L, eps: float, s: float, degree: int, p: int = 4):
+def cheb_inv_root(L, eps: float, s: float, degree: int, p: int = 4, prec=None):
     """X = s^{-1/p} sum_k c_k T_k(2 L/s - I)  ~  (L + s eps I)^{-1/p}."""
+    _, st = _model(prec)
     L = np.asarray(L, dtype=np.float64)
-    S = 2.0 * L / s - np.eye(L.shape[0])
-    P, mm = cheb_matrix(S, cheb_coefficients(degree, eps, p))
-    return s ** (-1.0 / p) * P, mm
+    S = st(2.0 * L / s - np.eye(L.shape[0]))
+    P, mm = cheb_matrix(S, cheb_coefficients(degree, eps, p), prec)
+    return s ** (-1.0 / p) * np.asarray(P, np.float64), mm
 
 
 def cheb_inv_root_replay(L, eps: float, s: float, degree: int, p: int = 4):

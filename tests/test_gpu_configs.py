@@ -1,0 +1,244 @@
+"""Parity on the five workload configurations.
+
+Inputs come from the seeded generators or from the oracle (float64, cast to
+float32); no input of a comparison is ever a GPU output.  Where the stack is
+too large for the oracle, outputs are compared on sampled matrices of the
+full-size launch.  Root tolerances: the stated 1e-3 (FP32) / 2e-2 (FP16
+coupled Newton), raised to three times what the same iteration reaches in
+IEEE float32 (or half) arithmetic when the input's conditioning puts the
+stated bound beyond any implementation in that precision
+(oracle.precision_floor).
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from matrix_roots_b200 import binding as B
+from matrix_roots_b200 import workloads as W
+from matrix_roots_b200.optimizer import BlockedShampoo, ShampooConfig
+
+from gpu_util import rel, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    assert torch.cuda.is_available()
+    from matrix_roots_b200 import build
+    build.build()
+    yield
+    assert B.device_error() == 0
+
+
+def _derived_tol(L, eps, s, method, iters, prec="fp32", stated=1e-3):
+    return max(stated, 3 * O.precision_floor(L, eps, s, method, iters, prec))
+
+
+# ------------------------------------------------------------- tiny dense ----
+
+def test_tiny_dense_ten_steps_match_evd_oracle():
+    """One 256x256 weight in 16 blocks of 64x64, 10 steps, beta2 = 1, NDB-20
+    FP32 on the GPU against float64 EVD roots in the oracle, SGD graft."""
+    import torch
+    G = W.tiny_dense_grads()
+    shapes = [(256, 256)]
+    cfg = ShampooConfig(block_size=64, beta2=1.0, alpha=1.0, eps=1e-6, method="ndb", iters=20, dtype="fp32",
+                        scaling="frobenius", graft="sgd", lr=0.1)
+    opt = BlockedShampoo(shapes, cfg)
+    Wd = [torch.zeros(256, 256, device="cuda")]
+    st = O.ShampooState(shapes, 64, "sgd")
+    Wr = [np.zeros((256, 256))]
+    for t in range(10):
+        opt.step(Wd, [to_dev(G[t])])
+        Wr = O.shampoo_step(st, Wr, [G[t]], beta2=1.0, alpha=1.0, eps=1e-6, method="evd", iters=0,
+                            scaling="frobenius", graft="sgd", lr=0.1)
+        err = rel(Wd[0].cpu().numpy(), Wr[0])
+        assert err < 1e-3, (t, err)
+    for f in range(len(st.factors)):
+        assert rel(opt.factors[f].cpu().numpy(), st.factors[f]) < 1e-5
+
+
+# ---------------------------------------------------------- low-rank stack ---
+
+def test_lowrank_stack_full():
+    """256 blocks of 128x128, G = U diag(1/i) V^T, 5 steps beta2 = 0.999;
+    NDB-15 and CN-15 FP32 with Frobenius scaling; direction; Adam graft."""
+    import torch
+    G = W.lowrank_stack_grads()
+    shapes = [(128, 128)] * 256
+    plan = B.Plan(shapes, 128).bind()
+    g_st = torch.empty((256, 128, 128), device="cuda")
+    F = torch.zeros((512, 128, 128), device="cuda")
+    for t in range(5):
+        B.stack_blocks(plan, [to_dev(G[t, i]) for i in range(256)], [g_st])
+        B.update_stats(plan, [g_st], [F], 0.999, 1.0, "fp32")
+    # oracle statistics (each block is its own layer: L_i at 2i? no: plan order)
+    ref_plan = O.plan_blocks(shapes, 128)
+    Lref = np.zeros((512, 128, 128))
+    for t in range(5):
+        for b in ref_plan["blocks"]:
+            gi, li, ri = int(b[8]), int(b[10]), int(b[12])
+            Lref[li], Lref[ri] = O.update_stats(G[t, gi], Lref[li], Lref[ri], 0.999)
+    Fh = F.cpu().numpy()
+    assert max(rel(Fh[i], Lref[i]) for i in range(512)) < 1e-5
+    # roots on the oracle's statistics
+    L32 = Lref.astype(np.float32)
+    roots = {}
+    for method in ("ndb", "cn"):
+        X, s, stt = B.inv_root(to_dev(L32), 1e-6, method, 15, "fp32", "frobenius")
+        X, s = X.cpu().numpy(), s.cpu().numpy()
+        assert int(np.abs(stt.cpu().numpy()).sum()) == 0
+        worst = 0.0
+        for i in range(0, 512, 7):
+            L = L32[i].astype(np.float64)
+            assert abs(s[i] / O.frobenius_scale(L, 1e-6) - 1) < 1e-5
+            worst = max(worst, rel(X[i], O.inv_root(L, 1e-6, method, 15, float(s[i]))))
+        assert worst < 1e-3, (method, worst)
+        roots[method] = X
+    # direction and Adam graft with the NDB roots (oracle: its own replayed roots)
+    Xd = to_dev(roots["ndb"])
+    d_st = torch.empty_like(g_st)
+    dn = torch.empty(256, device="cuda")
+    B.precondition(plan, [Xd], [g_st], [d_st], dn, "fp32")
+    Dh = d_st.cpu().numpy()
+    g_last = G[4]
+    sref = {i: O.frobenius_scale(L32[i].astype(np.float64), 1e-6) for i in range(512)}
+    worst = 0.0
+    for b in ref_plan["blocks"][::5]:
+        gi, li, ri = int(b[8]), int(b[10]), int(b[12])
+        XL = O.inv_root(L32[li].astype(np.float64), 1e-6, "ndb", 15, sref[li])
+        XR = O.inv_root(L32[ri].astype(np.float64), 1e-6, "ndb", 15, sref[ri])
+        worst = max(worst, rel(Dh[gi], O.precondition(XL, g_last[gi], XR)))
+    assert worst < 1e-3, worst
+
+
+# ------------------------------------------------------------- transformer ---
+
+def test_transformer_full_launch_sampled():
+    """8 layers d=1024, FFN 4096 at B=1024: 96 blocks / 192 factors of 1024^2.
+    Statistics of the whole stack against float64; NDB-20 FP32 with
+    power-iteration scaling on the oracle's statistics in the bench's launch
+    (count = 192), compared on sampled factors; the direction on sampled
+    blocks."""
+    import torch
+    shapes = W.transformer_shapes()
+    grads = W.transformer_grads(shapes, seed=0)
+    plan = B.Plan(shapes, 1024).bind()
+    t = plan.tables()
+    ref_plan = O.plan_blocks(shapes, 1024)
+    g_st = torch.empty((96, 1024, 1024), device="cuda")
+    F = torch.zeros((192, 1024, 1024), device="cuda")
+    B.stack_blocks(plan, [to_dev(g) for g in grads], [g_st])
+    B.update_stats(plan, [g_st], [F], 0.999, 1.0, "fp32")
+    G64 = O.stack_gradients(ref_plan, grads)[0]
+    assert np.array_equal(g_st.cpu().numpy(), G64.astype(np.float32))
+    Lref = np.empty((192, 1024, 1024), dtype=np.float32)
+    for b in ref_plan["blocks"]:
+        gi, li, ri = int(b[8]), int(b[10]), int(b[12])
+        L, R = O.update_stats(G64[gi], 0.0, 0.0, 0.999)
+        Lref[li], Lref[ri] = L, R
+    Fh = F.cpu().numpy()
+    for i in (0, 1, 95, 96, 150, 191):
+        assert rel(Fh[i], Lref[i]) < 1e-5
+    del Fh, F
+    starts = to_dev(W.power_iteration_starts(1024, 16))
+    X, s, stt = B.inv_root(to_dev(Lref), 1e-6, "ndb", 20, "fp32", "power", pi_vectors=16, pi_iters=10,
+                           pi_starts=starts)
+    assert int(np.abs(stt.cpu().numpy()).sum()) == 0
+    s = s.cpu().numpy()
+    errs = {}
+    for i in (0, 96, 191):
+        L = Lref[i].astype(np.float64)
+        lmax = np.linalg.eigvalsh(L)[-1] + 1e-6
+        assert 0.5 * lmax <= s[i] <= (1 + 1e-3) * lmax
+        ref = O.inv_root(L, 1e-6, "ndb", 20, float(s[i]))
+        err = rel(X[i].cpu().numpy(), ref)
+        tol = _derived_tol(L, 1e-6, float(s[i]), "ndb", 20)
+        errs[i] = (err, tol)
+        assert err < tol, (i, err, tol)
+    print("transformer NDB-20 FP32 root errors (err, bound):", errs)
+    d_st = torch.empty_like(g_st)
+    dn = torch.empty(96, device="cuda")
+    B.precondition(plan, [X], [g_st], [d_st], dn, "fp32")
+    for b in ref_plan["blocks"][[0, 40, 95]]:
+        gi, li, ri = int(b[8]), int(b[10]), int(b[12])
+        XL = O.inv_root(Lref[li].astype(np.float64), 1e-6, "ndb", 20, float(s[li]))
+        XR = O.inv_root(Lref[ri].astype(np.float64), 1e-6, "ndb", 20, float(s[ri]))
+        err = rel(d_st[gi].cpu().numpy(), O.precondition(XL, G64[gi], XR))
+        print("transformer direction block", gi, "rel err", err)
+        assert err < 1e-3
+
+
+# -------------------------------------------------------------- SPD stack ----
+
+SPD_CASES = [("cheb", 32, "fp32", 1e-3), ("cheb", 32, "fp16", 2e-2), ("ndb", 20, "fp32", 1e-3),
+             ("cn", 20, "fp16", 2e-2), ("cn", 20, "bf16", None)]
+
+
+@pytest.mark.parametrize("method,iters,dtype,stated", SPD_CASES)
+def test_spd_stack_methods(method, iters, dtype, stated):
+    """512 SPD 256x256 matrices, log-uniform spectrum in [1e-6, 1], eps = 1e-8,
+    Frobenius scaling; errors against the replay (parity) and against the
+    exact root (reported)."""
+    A32, Q, lam = W.spd_stack()
+    X, s, stt = B.inv_root(to_dev(A32), 1e-8, method, iters, dtype, "frobenius")
+    X, s, stt = X.cpu().numpy(), s.cpu().numpy(), stt.cpu().numpy()
+    rows = []
+    for i in (0, 77, 300, 511):
+        L = A32[i].astype(np.float64)
+        ref = O.inv_root(L, 1e-8, method, iters, float(s[i]))
+        exact = O.inv_root_exact(L, 1e-8)
+        err = rel(X[i], ref) if np.all(np.isfinite(X[i])) else float("inf")
+        rows.append((i, err, rel(ref, exact), rel(X[i], exact) if np.isfinite(err) else float("inf")))
+        if stated is not None:
+            tol = _derived_tol(L, 1e-8, float(s[i]), method, iters, dtype, stated)
+            assert err < tol, (i, err, tol)
+        else:
+            assert (stt[i] != 0) == (not np.all(np.isfinite(X[i])))
+    print(f"spd {method}-{iters} {dtype}: (matrix, err vs replay, method err vs exact, err vs exact)", rows)
+
+
+# ------------------------------------------------------------ large blocks ---
+
+def test_large_blocks_sampled():
+    """32 blocks of 2048x2048, rows scaled by exp(N(0,1)); EMA statistics
+    (beta2 = 0.999, 3 steps) on the GPU against float64 on sampled factors;
+    NDB-20 FP32 in a 64-factor launch on oracle statistics (8 distinct
+    factors repeated), compared on samples."""
+    import torch
+    G = W.large_block_grads()
+    shapes = [(2048, 2048)] * 32
+    plan = B.Plan(shapes, 2048).bind()
+    ref_plan = O.plan_blocks(shapes, 2048)
+    g_st = torch.empty((32, 2048, 2048), device="cuda")
+    F = torch.zeros((64, 2048, 2048), device="cuda")
+    for t in range(3):
+        B.stack_blocks(plan, [to_dev(G[t, i]) for i in range(32)], [g_st])
+        B.update_stats(plan, [g_st], [F], 0.999, 0.001, "fp32")
+    sample_blocks = [0, 5, 31]
+    Lref = {}
+    for b in ref_plan["blocks"][sample_blocks]:
+        gi, li, ri = int(b[8]), int(b[10]), int(b[12])
+        L, R = np.zeros((2048, 2048)), np.zeros((2048, 2048))
+        for t in range(3):
+            L, R = O.update_stats(G[t, gi], L, R, 0.999, 0.001)
+        Lref[li], Lref[ri] = L, R
+        assert rel(F[li].cpu().numpy(), L) < 1e-5
+        assert rel(F[ri].cpu().numpy(), R) < 1e-5
+    del F
+    keys = sorted(Lref)[:6] + sorted(Lref)[:2]
+    stack = np.stack([Lref[k].astype(np.float32) for k in keys] * 8)
+    X, s, stt = B.inv_root(to_dev(stack), 1e-6, "ndb", 20, "fp32", "frobenius")
+    assert int(np.abs(stt.cpu().numpy()).sum()) == 0
+    s = s.cpu().numpy()
+    Xh = {i: X[i].cpu().numpy() for i in (0, 8, 61)}
+    assert np.array_equal(Xh[0], Xh[8])  # same input matrix, same result anywhere in the launch
+    for i in (0, 61):
+        L = stack[i].astype(np.float64)
+        ref = O.inv_root(L, 1e-6, "ndb", 20, float(s[i]))
+        err = rel(Xh[i], ref)
+        tol = _derived_tol(L, 1e-6, float(s[i]), "ndb", 20)
+        print("large-block NDB root", i, "err", err, "bound", tol)
+        assert err < tol

@@ -370,6 +370,37 @@ def test_cheb_high_degree_reaches_damped_root():
     assert O.rel_fro(X, O.inv_root_exact(L, 0.05 * s)) < 1e-10
 
 
+# ---------------------------------------------------------------- models -------
+
+def test_round_mantissa_matches_ieee_half():
+    # fp16 keeps 10 explicit mantissa bits: inside its normal range, rounding
+    # a float32 to 10 bits (ties to even) is exactly numpy's half conversion
+    rng = np.random.default_rng(30)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-8, 8, 20000))).astype(np.float32)
+    x = x[(np.abs(x) > 6.2e-5) & (np.abs(x) < 6.0e4)]
+    assert np.array_equal(O.round_mantissa(x, 10), x.astype(np.float16).astype(np.float32))
+
+
+def test_truncate_mantissa_values():
+    one = np.float32(1.0)
+    u = np.float32(2.0 ** -10)
+    x = np.array([1 + 2 ** -11 + 2 ** -12, 1 + u + 2 ** -11, -(1 + u - 2 ** -12), 3.0], dtype=np.float32)
+    assert list(O.truncate_mantissa(x, 10)) == [one, one + u, -one, np.float32(3.0)]
+    y = np.random.default_rng(31).standard_normal(1000).astype(np.float32)
+    t = O.truncate_mantissa(y, 10)
+    assert np.all(np.abs(t) <= np.abs(y)) and np.all(np.abs(y - t) < np.abs(y) * 2.0 ** -10)
+
+
+def test_precision_models_bracket_exact_result():
+    rng = np.random.default_rng(32)
+    L, _, _ = _spd(rng, 24, cond=50.0)
+    s = O.frobenius_scale(L, 1e-3)
+    e32 = O.precision_floor(L, 1e-3, s, "ndb", 10, "fp32")
+    e16 = O.precision_floor(L, 1e-3, s, "ndb", 10, "fp16")
+    ebf = O.precision_floor(L, 1e-3, s, "ndb", 10, "bf16")
+    assert e32 < 1e-5 < e16 < ebf < 1e-1
+
+
 # ---------------------------------------------------------------- O5 -----------
 
 def test_direction_frobenius_bounds():

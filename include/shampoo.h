@@ -192,6 +192,33 @@ SHP_API shp_status shampoo_inv_root(const float* A, int32_t count, int32_t n, fl
                             const float* pi_starts, float* X_out, float* scale_out, int32_t* status_out,
                             void* workspace, size_t ws_bytes, void* stream);
 
+/* Bytes of device scratch behind shampoo_inv_root_static (32 MiB). */
+#define SHP_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* shampoo_inv_root for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is a property of the library, not of the
+ * method.  Callers that cannot call cudaMalloc at the moment they need a
+ * root -- code running while a CUDA graph is captured, allocator or
+ * memory-pool callbacks that must not re-enter the allocator, programs with
+ * a fixed preallocated memory budget -- get the same result as
+ * shampoo_inv_root (same arguments minus the workspace) with the scratch
+ * taken from a device array of SHP_STATIC_SCRATCH_BYTES that the library
+ * defines.  Every GPU that loads this part of the library holds that array
+ * until the process exits.
+ *   - Rejects (SHP_ERR_WORKSPACE, nothing enqueued) any request whose
+ *     shampoo_inv_root_workspace_bytes exceeds SHP_STATIC_SCRATCH_BYTES.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Calls no cudaMalloc / cudaFree and no allocating library routine.
+ *   - All calls on a device share the one array and it keeps the last
+ *     call's contents (everything a call reads is written by that call
+ *     first); calls whose work overlaps on the GPU (different streams
+ *     without ordering) race on it. */
+SHP_API shp_status shampoo_inv_root_static(const float* A, int32_t count, int32_t n, float eps, int32_t p,
+                                           int32_t method, int32_t iters, int32_t dtype, int32_t scaling,
+                                           int32_t pi_vectors, int32_t pi_iters, const float* pi_starts,
+                                           float* X_out, float* scale_out, int32_t* status_out, void* stream);
+
 /* ---------------------------------------------------------------------
  * a7  Two-sided preconditioning   ([DASH] §2)
  *   D_b = X_L(b) G_b X_R(b)   for every gradient block b

@@ -26,7 +26,7 @@ EXPORTS = [
     "shampoo_plan_create", "shampoo_plan_destroy", "shampoo_plan_sizes", "shampoo_plan_tables",
     "shampoo_plan_bind", "shampoo_stack_blocks",
     "shampoo_update_stats_workspace_bytes", "shampoo_update_stats",
-    "shampoo_inv_root_workspace_bytes", "shampoo_inv_root",
+    "shampoo_inv_root_workspace_bytes", "shampoo_inv_root", "shampoo_inv_root_static",
     "shampoo_precondition_workspace_bytes", "shampoo_precondition",
     "shampoo_graft_step_workspace_bytes", "shampoo_graft_step",
 ]
@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         "shampoo_inv_root": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_int32, c_int32, c_int32, c_int32,
                                        c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_size_t, c_void_p]),
+        "shampoo_inv_root_static": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_int32, c_int32, c_int32,
+                                              c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_void_p]),
         "shampoo_precondition_workspace_bytes": (c_size_t, [c_void_p, c_int32]),
         "shampoo_precondition": (c_int32, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), c_void_p, c_int32,
                                            c_void_p, c_size_t, c_void_p]),
@@ -216,6 +219,26 @@ def inv_root(A, eps: float, method="ndb", iters: int = 20, dtype="fp32", scaling
                                   _enum(DTYPES, dtype), _enum(SCALINGS, scaling), int(pi_vectors), int(pi_iters),
                                   _ptr(pi_starts), _ptr(X), _ptr(s), _ptr(st), _ptr(workspace), workspace.numel(),
                                   _stream(stream)), "shampoo_inv_root")
+    return X, s, st
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def inv_root_static(A, eps: float, method="ndb", iters: int = 20, dtype="fp32", scaling="frobenius", p: int = 4,
+                    pi_vectors: int = 16, pi_iters: int = 10, pi_starts=None, out=None, scale_out=None,
+                    status_out=None, stream=None):
+    """shampoo_inv_root_static: same as inv_root, scratch from the library's
+    fixed device array (for callers that cannot allocate); returns (X, scale, status)."""
+    import torch
+    count, n = int(A.shape[0]), int(A.shape[1])
+    X = out if out is not None else torch.empty_like(A)
+    s = scale_out if scale_out is not None else torch.empty(count, dtype=torch.float32, device=A.device)
+    st = status_out if status_out is not None else torch.empty(count, dtype=torch.int32, device=A.device)
+    _check(lib().shampoo_inv_root_static(_ptr(A), count, n, float(eps), int(p), _enum(METHODS, method), int(iters),
+                                         _enum(DTYPES, dtype), _enum(SCALINGS, scaling), int(pi_vectors),
+                                         int(pi_iters), _ptr(pi_starts), _ptr(X), _ptr(s), _ptr(st),
+                                         _stream(stream)), "shampoo_inv_root_static")
     return X, s, st
 
 

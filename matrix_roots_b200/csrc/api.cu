@@ -427,6 +427,8 @@ LayerArgs layer_args(const shp_plan* plan, int l0, int l1, float* const* W, cons
 
 }  // namespace
 
+void shp::set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 // ============================================================================
 extern "C" {
 

@@ -120,4 +120,7 @@ unsigned long long launch_total();
 // Reads and clears the device error word (synchronous).
 cudaError_t read_and_clear_dev_error(int* out);
 
+// Sets the calling thread's shampoo_last_error() message.
+void set_last_error(const char* msg);
+
 }  // namespace shp

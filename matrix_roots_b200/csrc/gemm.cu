@@ -289,6 +289,340 @@ __global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ Ge
   }
 }
 
+// ---- FP32 (3 x TF32) persistent kernel with drained accumulation ----------
+//
+// The tensor core's FP32 accumulation error grows with the number of
+// products chained into one accumulator.  Here each K-block (32 deep, 12
+// MMAs: lo*hi, hi*lo, hi*hi over 4 slices) goes into its own slot of a
+// 4-deep TMEM ring; accumulator warps drain every slot into fp32 registers
+// (round to nearest) and release it.  Two accumulator warpgroups take
+// alternate tiles, so one runs a tile's epilogue while the other drains the
+// next tile.  One CTA per SM walks the tiles of all matrices (persistent).
+//   warps 0-7  accumulator warpgroups (warp w reads TMEM lanes 32*(w%4)..)
+//   warp 8     TMEM allocator + single-thread MMA issuer
+//   warp 9     single-thread TMA producer
+
+template <int BN>
+struct Cfg3 {
+  static constexpr int A_TILE = 128 * 128;
+  static constexpr int B_TILE = BN * 128;
+  static constexpr int STAGE_BYTES = 2 * (A_TILE + B_TILE);  // hi and lo planes
+  static constexpr int STAGES_RAW = (227 * 1024 - 4096) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
+  static constexpr int NBUF = 4;
+  static constexpr int TCOLS = NBUF * BN;
+  static constexpr int THREADS = 320;
+  static constexpr int STAGE_OUT = 8 * 32 * 32 * 4;  // 32x32 transpose buffer per draining warp
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512 + STAGE_OUT;
+  static_assert(STAGES >= 2 && TCOLS <= 512, "FP32 tile does not fit");
+  static_assert(SMEM_BYTES <= 227 * 1024, "FP32 tile does not fit");
+};
+
+// Epilogue of a 32-row x 32-column block whose accumulators sit transposed
+// in `stage` (element (r, c) at r*32 + (c ^ r)): lane = column, so every
+// load of C and every store of an output plane is one 128-byte segment.
+__device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row0, int col, const float* stage,
+                                               int lane, float& ss, int& bad) {
+  const int ob = g.o_idx ? g.o_idx[b] : b;
+  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
+  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
+  if (col >= g.N) return;
+  long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
+  long long ooff = (long long)ob * g.O.bs + (long long)row0 * g.O.ld + col;
+  long long xoff = (long long)ob * g.X.bs + (long long)row0 * g.X.ld + col;
+  const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
+  for (int r = 0; r < rmax; ++r, coff += g.C.ld, ooff += g.O.ld, xoff += g.X.ld) {
+    const float a = stage[r * 32 + (lane ^ r)];
+    float cval = 0.f;
+    if (need_c) {
+      cval = g.C.f32[coff];
+      if (g.C.lo) cval += g.C.lo[coff];
+    }
+    const float diag = (row0 + r == col) ? 1.f : 0.f;
+    const float r0 = g.alpha * a + g.beta * cval + g.gamma * diag;
+    const float v = r0 * mult;
+    write_out(g.O, ooff, v);
+    ss += v * v;
+    bad |= !isfinite(v);
+    if (has_x) write_out(g.X, xoff, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
+  }
+}
+
+struct Tile {
+  int grp, b, m0, n0, nk;
+};
+
+__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN) {
+  Tile x;
+  x.grp = t >= p.tiles0 ? 1 : 0;
+  int r = x.grp ? t - p.tiles0 : t;
+  const int per = p.mt[x.grp] * p.nt[x.grp];
+  x.b = r / per;
+  r -= x.b * per;
+  const int mi = r / p.nt[x.grp];
+  x.m0 = mi * 128;
+  x.n0 = (r - mi * p.nt[x.grp]) * BN;
+  x.nk = (p.g[x.grp].K + 31) / 32;
+  return x;
+}
+
+// Fused epilogue of one accumulator row held in registers; returns sum r^2.
+template <int BN>
+__device__ __forceinline__ float epilogue_row(const GroupDev& g, int b, int row, int n0, const float (&acc)[BN],
+                                              int& bad) {
+  if (row >= g.M) return 0.f;
+  const int ob = g.o_idx ? g.o_idx[b] : b;
+  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
+  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
+  const long long crow = (long long)ob * g.C.bs + (long long)row * g.C.ld;
+  const long long orow = (long long)ob * g.O.bs + (long long)row * g.O.ld;
+  const long long xrow = (long long)ob * g.X.bs + (long long)row * g.X.ld;
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < BN; c += 16) {
+    if (n0 + c < g.N) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int col = n0 + c + i;
+        if (col < g.N) {
+          float cval = 0.f;
+          if (need_c) {
+            cval = g.C.f32[crow + col];
+            if (g.C.lo) cval += g.C.lo[crow + col];
+          }
+          const float diag = (row == col) ? 1.f : 0.f;
+          const float r0 = g.alpha * acc[c + i] + g.beta * cval + g.gamma * diag;
+          const float r = r0 * mult;
+          write_out(g.O, orow + col, r);
+          ss += r * r;
+          bad |= !isfinite(r);
+          if (has_x) write_out(g.X, xrow + col, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
+        }
+      }
+    }
+  }
+  return ss;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg3<BN>;
+  constexpr int S = C::STAGES;
+  constexpr int NB = C::NBUF;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3 * NB);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * S;
+  const uint32_t tfull0 = empty0 + 8 * S;       // [NB] slot written by the MMA
+  const uint32_t tempty0 = tfull0 + 8 * 2 * NB;  // [NB] slot drained by both groups
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int j = 0; j < NB; ++j) {
+      mbar_init(tfull0 + 8 * j, 1);
+      mbar_init(tempty0 + 8 * j, 256);  // every thread of both draining warpgroups
+    }
+    // skip all tiles once any CTA has given up on a barrier
+    *abort_flag = (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) ? 1 : 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), C::TCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = p.total_tiles;
+
+  if (warp == 9) {
+    if (lane == 0) {
+      uint32_t gs = 0;
+      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const Tile x = decode_tile(p, t, BN);
+        const GroupDev& g = p.g[x.grp];
+        const int ab = g.a_idx ? g.a_idx[x.b] : x.b;
+        const int bb = g.b_idx ? g.b_idx[x.b] : x.b;
+        for (int kb = 0; kb < x.nk; ++kb, ++gs) {
+          const int s = gs % S;
+          if (gs >= S && !mbar_wait(empty0 + 8 * s, ((gs / S) - 1) & 1)) {
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * s;
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          const int k0 = kb * 32;
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+#pragma unroll
+          for (int pl = 0; pl < 2; ++pl) {
+            const CUtensorMap* ma = &p.tmA[x.grp][pl];
+            const CUtensorMap* mb = &p.tmB[x.grp][pl];
+            const uint32_t sa = smem_u32(st + pl * C::A_TILE);
+            const uint32_t sb = smem_u32(st + 2 * C::A_TILE + pl * C::B_TILE);
+            if (!g.a_mn) {
+              tma_load_3d(sa, ma, fb, k0, x.m0, ab);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) tma_load_3d(sa + j * 4096, ma, fb, x.m0 + j * 32, k0, ab);
+            }
+            if (!g.b_mn) {
+              tma_load_3d(sb, mb, fb, k0, x.n0, bb);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 32; ++j) tma_load_3d(sb + j * 4096, mb, fb, x.n0 + j * 32, k0, bb);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 8) {
+    if (lane == 0) {
+      uint32_t gs = 0, gk = 0;
+      for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+        const Tile x = decode_tile(p, t, BN);
+        const GroupDev& g = p.g[x.grp];
+        const uint32_t idesc = idesc_f32acc(2, 2, g.a_mn, g.b_mn, 128, BN);
+        const uint32_t a_step = g.a_mn ? 1024u : 32u, b_step = g.b_mn ? 1024u : 32u;
+        const uint32_t a_lbo = g.a_mn ? 4096u : 16u, b_lbo = g.b_mn ? 4096u : 16u;
+        const uint32_t a_sbo = g.a_mn ? 512u : 1024u, b_sbo = g.b_mn ? 512u : 1024u;
+        const uint32_t a_lay = g.a_mn ? 1u : 2u, b_lay = g.b_mn ? 1u : 2u;
+        for (int kb = 0; kb < x.nk; ++kb, ++gs, ++gk) {
+          const int s = gs % S;
+          const int j = gk % NB;
+          if (!mbar_wait(full0 + 8 * s, (gs / S) & 1) ||
+              (gk >= NB && !mbar_wait(tempty0 + 8 * j, ((gk / NB) - 1) & 1))) {
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const uint32_t sa0 = smem_u32(st), sb0 = smem_u32(st + 2 * C::A_TILE);
+          const uint32_t d = tmem + (uint32_t)(j * BN);
+          // the 8 small correction products first, while the accumulator is
+          // small, then the 4 hi*hi products: only those 4 additions happen
+          // at the scale of the full partial sum
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
+            const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
+            mma_tf32(d, a_lo, b_hi, idesc, ks ? 1u : 0u);
+            mma_tf32(d, a_hi, b_lo, idesc, 1u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
+            mma_tf32(d, a_hi, b_hi, idesc, 1u);
+          }
+          tc_commit(empty0 + 8 * s);
+          tc_commit(tfull0 + 8 * j);
+        }
+      }
+    }
+  } else {
+    // both warpgroups drain every K-block; group h owns columns
+    // [h*BN/2, (h+1)*BN/2) of the tile, warp w%4 owns TMEM lanes 32*(w%4)..
+    constexpr int HC = BN / 2;
+    const int h = warp >> 2;
+    const int q = warp & 3;
+    uint32_t gk = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (*abort_flag) break;
+      const Tile x = decode_tile(p, t, BN);
+      float acc[HC];
+#pragma unroll
+      for (int i = 0; i < HC; ++i) acc[i] = 0.f;
+      bool ok = true;
+      for (int kb = 0; kb < x.nk; ++kb, ++gk) {
+        const int j = gk % NB;
+        ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * j, (gk / NB) & 1));
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r[HC];
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(j * BN + h * HC);
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) tmem_ld32_nowait(base + c, r + c);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < HC; ++i) acc[i] += __uint_as_float(r[i]);
+        tc_fence_before();
+        mbar_arrive(tempty0 + 8 * j);
+      }
+      if (!ok) break;
+      const GroupDev& g = p.g[x.grp];
+      int bad = 0;
+      float ss = 0.f;
+      float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + warp * 1024;
+#pragma unroll
+      for (int ch = 0; ch < HC / 32; ++ch) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = acc[ch * 32 + c];
+        __syncwarp();
+        epilogue_block(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad);
+        __syncwarp();
+      }
+      if (g.sumsq) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) atomicAdd(g.sumsq + (g.o_idx ? g.o_idx[x.b] : x.b), ss);
+      }
+      if (g.status && bad) atomicOr(g.status + (g.o_idx ? g.o_idx[x.b] : x.b), 1);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TCOLS);
+  }
+}
+
+int num_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
+template <int BN>
+cudaError_t run3(GemmParams& prm, cudaStream_t stream) {
+  using C = Cfg3<BN>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm3_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
+  gemm3_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---- host side -------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -391,9 +725,19 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
         return cudaErrorInvalidValue;
     }
   }
-  if (kind == 0 && npass == 3) {
-    if (BN == 64) return run<0, 3, 64>(prm, ngroups, batch, maxM, maxN, stream);
-    return run<0, 3, 128>(prm, ngroups, batch, maxM, maxN, stream);
+  if (kind == 0 && npass == 3) {  // persistent kernel over all tiles of all matrices
+    long long total = 0;
+    for (int i = 0; i < ngroups; ++i) {
+      prm.mt[i] = (groups[i].M + 127) / 128;
+      prm.nt[i] = (groups[i].N + BN - 1) / BN;
+      const long long ti = (long long)batch * prm.mt[i] * prm.nt[i];
+      if (i == 0) prm.tiles0 = (int)ti;
+      total += ti;
+    }
+    if (total > (1ll << 30)) return cudaErrorInvalidValue;
+    prm.total_tiles = (int)total;
+    if (BN == 64) return run3<64>(prm, stream);
+    return run3<128>(prm, stream);
   }
   if (kind == 0) {
     if (BN == 64) return run<0, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);

@@ -69,6 +69,10 @@ struct alignas(64) GemmParams {
   GroupDev g[2];
   int ngroups;
   int batch;
+  // persistent schedule: tiles of group 0 (batch x mt x nt, matrix-major)
+  // come first, then group 1
+  int mt[2], nt[2];
+  int tiles0, total_tiles;
 };
 
 // Host description of one group before tensor maps are built.

@@ -489,8 +489,12 @@ def cheb_inv_root_replay(L, eps: float, s: float, degree: int, p: int = 4):
     return (Q * (s ** (-1.0 / p) * x)) @ Q.T
 
 
-def inv_root(L, eps: float, method: str, iters: int, scale: float, p: int = 4, replay: bool = True):
-    """Dispatch to the method (eigenvalue replay when ``replay``)."""
+def inv_root(L, eps: float, method: str, iters: int, scale: float, p: int = 4, replay: bool = True, prec=None):
+    """Dispatch to the method (eigenvalue replay when ``replay``; the matrix
+    form in arithmetic model ``prec`` when one is given)."""
+    if prec is not None and method != "evd":
+        fn = {"ndb": ndb_inv_root, "cn": cn_inv_root, "cheb": cheb_inv_root}[method]
+        return fn(L, eps, scale, iters, prec=prec)[0] if method == "ndb" else fn(L, eps, scale, iters, p, prec)[0]
     if method == "ndb":
         return ndb_inv_root_replay(L, eps, scale, iters) if replay else ndb_inv_root(L, eps, scale, iters)[0]
     if method == "cn":
@@ -587,7 +591,7 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
                  method: str, iters: int, scaling: str, graft: str, lr: float,
                  beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
                  wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
-                 replay: bool = True):
+                 replay: bool = True, prec=None):
     """One optimizer step over all layers; returns the new weights.
 
     ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
@@ -600,6 +604,8 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
         state.factors[lb][lix], state.factors[rb][rix] = update_stats(
             g_st[gb][gi], state.factors[lb][lix], state.factors[rb][rix], beta2, alpha)
+    if prec is not None:  # the arithmetic model also stores the statistics in float32
+        state.factors = [f.astype(np.float32).astype(np.float64) for f in state.factors]
     roots = [np.empty_like(f) for f in state.factors]
     for fb, stack in enumerate(state.factors):
         for i in range(stack.shape[0]):
@@ -612,7 +618,7 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
                 s = power_iteration_scale(Lf, 0.0 if method == "cheb" else eps, pi_starts, pi_iters)
             if scales_out is not None:
                 scales_out[(fb, i)] = s
-            roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay)
+            roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay, prec=prec)
     d_st = [np.empty_like(g) for g in g_st]
     for b in plan["blocks"]:
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])

@@ -393,8 +393,35 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+def run_root_stack(args):
+    """Small fixed case of the dominant kernel for profilers: Newton-DB-20
+    on `args.root_stack` factors L = G G^T of transformer gradient blocks
+    (1024^2), two shampoo_inv_root calls; prints one JSON line."""
+    import torch
+    from matrix_roots_b200 import binding as B
+    from matrix_roots_b200 import build
+    from matrix_roots_b200 import workloads as W
+    build.build()
+    k = args.root_stack
+    g = W.transformer_grads([(1024, 1024)] * k, seed=0)
+    L = np.stack([(x.astype(np.float64) @ x.astype(np.float64).T).astype(np.float32) for x in g])
+    A = torch.from_numpy(L).cuda()
+    ws = torch.empty(B.inv_root_workspace_bytes(k, 1024, "ndb", args.dtype, "frobenius"), dtype=torch.uint8,
+                     device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    B.inv_root(A, 1e-6, "ndb", 20, args.dtype, "frobenius", workspace=ws)
+    e0.record()
+    X, s, st = B.inv_root(A, 1e-6, "ndb", 20, args.dtype, "frobenius", workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    assert B.device_error() == 0 and int(st.abs().sum()) == 0
+    print(json.dumps({"case": f"ndb20_{args.dtype}_{k}x1024", "ms": e0.elapsed_time(e1)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--root-stack", type=int, default=0,
+                    help="profile case: Newton-DB roots of this many 1024^2 factors, then exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -406,6 +433,9 @@ def main():
     ap.add_argument("--cpu-blocks", type=int, default=4)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.root_stack:
+        run_root_stack(args)
+        return
     cfg = CONFIGS[args.config]
     if args.impl == "reference":
         run_reference(args, cfg)

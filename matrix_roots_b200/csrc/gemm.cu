@@ -4,14 +4,23 @@
 // and Efficient Inverse-Root Solvers", §4: same-shape blocks stacked into 3D
 // tensors and processed by batched matmuls).
 //
-// One CTA computes a 128 x BN tile of one matrix of the stack:
-//   warp 5      TMA producer: 128B-swizzled operand tiles into a STAGES-deep
+// One persistent CTA per SM walks the 128 x BN output tiles of every matrix
+// of the stack (and of up to two problems per launch):
+//   warp 9      TMA producer: 128B-swizzled operand tiles into a STAGES-deep
 //               shared-memory ring (mbarrier complete_tx)
-//   warp 4      TMEM allocator + single-thread tcgen05.mma issuer; FP32 mode
-//               issues lo*hi + hi*lo + hi*hi (3 x TF32) per K step
-//   warps 0..3  epilogue: tcgen05.ld of the FP32 accumulator, the fused
-//               a*D + b*C + c*I combination, norm / finiteness reductions
-//               and the plane writes the next GEMM reads.
+//   warp 8      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 0-7   two draining warpgroups (warp w reads TMEM lanes 32*(w%4)..,
+//               group h owns columns [h*BN/2, (h+1)*BN/2) of the tile)
+// The tensor core's FP32 accumulation error grows with the number of
+// products chained into one accumulator, so each K-block (one 128-byte row
+// of K: 32 tf32 or 64 f16/bf16 elements, 4 MMA slices) goes into its own
+// slot of a 4-deep TMEM ring; the draining warps add every slot into fp32
+// registers (round to nearest) and release it.  In FP32 mode (three TF32
+// passes on hi/lo operand splits) the small correction products lo*hi and
+// hi*lo are issued before hi*hi, so only the 4 hi*hi additions of a K-block
+// happen at the scale of the full partial sum.  The epilogue transposes
+// 32x32 blocks through shared memory so that reads of C and writes of the
+// output planes are 128-byte coalesced.
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -43,40 +52,51 @@ cudaError_t read_and_clear_dev_error(int* out) {
 
 namespace {
 
+// MMA kind: 0 = tf32, 1 = f16, 2 = bf16 (all with FP32 accumulation).
 template <int KIND>
 struct KindTraits;
 template <>
-struct KindTraits<0> {  // tf32
+struct KindTraits<0> {
   static constexpr int ESZ = 4;
   static constexpr uint32_t FMT = 2;
   static constexpr int KINST = 8;
+  // MN-major tf32 tiles: 128B swizzle with 32-byte atoms (UMMA layout 1,
+  // 4-row atoms of 512 B), the only MN-major layout the tensor core accepts
+  // for 32-bit operands
+  static constexpr uint32_t MN_LAYOUT = 1, MN_SBO = 512;
 };
 template <>
-struct KindTraits<1> {  // f16
+struct KindTraits<1> {
   static constexpr int ESZ = 2;
   static constexpr uint32_t FMT = 0;
   static constexpr int KINST = 16;
+  static constexpr uint32_t MN_LAYOUT = 2, MN_SBO = 1024;
 };
 template <>
-struct KindTraits<2> {  // bf16
+struct KindTraits<2> {
   static constexpr int ESZ = 2;
   static constexpr uint32_t FMT = 1;
   static constexpr int KINST = 16;
+  static constexpr uint32_t MN_LAYOUT = 2, MN_SBO = 1024;
 };
 
 template <int KIND, int NPASS, int BN>
 struct Cfg {
-  static constexpr int NPL = (NPASS == 3) ? 2 : 1;
   static constexpr int ESZ = KindTraits<KIND>::ESZ;
-  static constexpr int BKE = 128 / ESZ;  // K elements per stage (one 128-byte swizzle row)
+  static constexpr int BKE = 128 / ESZ;  // K elements per K-block (one 128-byte swizzle row)
+  static constexpr int NPL = (NPASS == 3) ? 2 : 1;
   static constexpr int A_TILE = 128 * 128;
   static constexpr int B_TILE = BN * 128;
   static constexpr int STAGE_BYTES = NPL * (A_TILE + B_TILE);
-  static constexpr int SMEM_BUDGET = 227 * 1024 - 2048;
-  static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static_assert(STAGES >= 2, "tile does not fit shared memory");
+  static constexpr int NBUF = 4;
+  static constexpr int TCOLS = NBUF * BN;
+  static constexpr int THREADS = 320;
+  static constexpr int STAGE_OUT = 8 * 32 * 32 * 4;  // 32x32 transpose buffer per draining warp
+  static constexpr int RESERVED = 1024 + 512 + STAGE_OUT;
+  static constexpr int STAGES_RAW = (227 * 1024 - RESERVED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RESERVED;
+  static_assert(STAGES >= 2 && TCOLS <= 512 && BN <= 128, "tile does not fit");
 };
 
 __device__ __forceinline__ void store_h16(void* base, long long off, float v, int bf) {
@@ -97,226 +117,23 @@ __device__ __forceinline__ void write_out(const EpiOut& o, long long off, float 
   if (o.h16) store_h16(o.h16, off, r, o.h16_bf);
 }
 
-template <int KIND, int NPASS, int BN>
-__global__ void __launch_bounds__(192, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<KIND, NPASS, BN>;
-  constexpr int STAGES = C::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int z = blockIdx.z;
-  const int grp = z / p.batch;
-  const int b = z - grp * p.batch;
-  const GroupDev& g = p.g[grp];
-  const int m0 = blockIdx.y * 128;
-  const int n0 = blockIdx.x * BN;
-  if (m0 >= g.M || n0 >= g.N) return;  // uniform for the whole CTA
-  // once any CTA has given up on a barrier, later CTAs skip their tile
-  // instead of each waiting out its own time limit
-  if (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) return;
-  const int nk = (g.K + C::BKE - 1) / C::BKE;
-
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + STAGES);
-  const uint32_t accum_bar = smem_u32(bars + 2 * STAGES);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    mbar_init(accum_bar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 4) {
-    tmem_alloc(smem_u32(tmem_slot), BN);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 5) {
-    if (lane == 0) {
-      const CUtensorMap* mA0 = &p.tmA[grp][0];
-      const CUtensorMap* mA1 = &p.tmA[grp][1];
-      const CUtensorMap* mB0 = &p.tmB[grp][0];
-      const CUtensorMap* mB1 = &p.tmB[grp][1];
-      const int ab = g.a_idx ? g.a_idx[b] : b;
-      const int bb = g.b_idx ? g.b_idx[b] : b;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        if (kb >= STAGES && !mbar_wait(empty0 + 8 * s, ((kb / STAGES) - 1) & 1)) {
-          *abort_flag = 1;
-          break;
-        }
-        const uint32_t fb = full0 + 8 * s;
-        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-        const int k0 = kb * C::BKE;
-        uint8_t* st = smem + s * C::STAGE_BYTES;
-#pragma unroll
-        for (int pl = 0; pl < C::NPL; ++pl) {
-          const CUtensorMap* ma = pl ? mA1 : mA0;
-          const CUtensorMap* mb = pl ? mB1 : mB0;
-          const uint32_t sa = smem_u32(st + pl * C::A_TILE);
-          const uint32_t sb = smem_u32(st + C::NPL * C::A_TILE + pl * C::B_TILE);
-          if (!g.a_mn) {
-            tma_load_3d(sa, ma, fb, k0, m0, ab);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 128 / C::BKE; ++j) tma_load_3d(sa + j * C::BKE * 128, ma, fb, m0 + j * C::BKE, k0, ab);
-          }
-          if (!g.b_mn) {
-            tma_load_3d(sb, mb, fb, k0, n0, bb);
-          } else {
-#pragma unroll
-            for (int j = 0; j < BN / C::BKE; ++j) tma_load_3d(sb + j * C::BKE * 128, mb, fb, n0 + j * C::BKE, k0, bb);
-          }
-        }
-      }
-    }
-  } else if (warp == 4) {
-    if (lane == 0) {
-      constexpr uint32_t FMT = KindTraits<KIND>::FMT;
-      const uint32_t idesc = idesc_f32acc(FMT, FMT, g.a_mn, g.b_mn, 128, BN);
-      // byte step of one MMA K-slice inside a stage, per operand major-ness
-      constexpr uint32_t KSTEP_K = KindTraits<KIND>::KINST * C::ESZ;  // 32 bytes
-      constexpr uint32_t KSTEP_MN = KindTraits<KIND>::KINST * 128;     // KINST rows of 128 bytes
-      constexpr uint32_t LBO_MN = C::BKE * 128;                          // one TMA box along M/N
-      const uint32_t a_step = g.a_mn ? KSTEP_MN : KSTEP_K;
-      const uint32_t b_step = g.b_mn ? KSTEP_MN : KSTEP_K;
-      const uint32_t a_lbo = g.a_mn ? LBO_MN : 16u;
-      const uint32_t b_lbo = g.b_mn ? LBO_MN : 16u;
-      // MN-major tf32 tiles use the 32-byte-atom swizzle (4-row atoms, 512 B)
-      constexpr bool MN32 = (KIND == 0);
-      const uint32_t a_lay = (g.a_mn && MN32) ? 1u : 2u;
-      const uint32_t b_lay = (g.b_mn && MN32) ? 1u : 2u;
-      const uint32_t a_sbo = (g.a_mn && MN32) ? 512u : 1024u;
-      const uint32_t b_sbo = (g.b_mn && MN32) ? 512u : 1024u;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(full0 + 8 * s, (kb / STAGES) & 1)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        uint8_t* st = smem + s * C::STAGE_BYTES;
-        const uint32_t sa0 = smem_u32(st);
-        const uint32_t sb0 = smem_u32(st + C::NPL * C::A_TILE);
-#pragma unroll
-        for (int ks = 0; ks < C::BKE / KindTraits<KIND>::KINST; ++ks) {
-          const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
-          const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
-          const uint32_t acc = (kb | ks) ? 1u : 0u;
-          if constexpr (NPASS == 3) {
-            const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
-            const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
-            mma_tf32(tmem, a_lo, b_hi, idesc, acc);
-            mma_tf32(tmem, a_hi, b_lo, idesc, 1u);
-            mma_tf32(tmem, a_hi, b_hi, idesc, 1u);
-          } else if constexpr (KIND == 0) {
-            mma_tf32(tmem, a_hi, b_hi, idesc, acc);
-          } else {
-            mma_f16(tmem, a_hi, b_hi, idesc, acc);
-          }
-        }
-        tc_commit(empty0 + 8 * s);
-      }
-      tc_commit(accum_bar);  // also on abort, so the epilogue never waits forever
-    }
-  } else {
-    // ---------------- epilogue: warps 0..3, thread <-> accumulator row ----
-    const bool ok = mbar_wait(accum_bar, 0);
-    tc_fence_after();
-    __syncwarp();
-    if (ok && !*abort_flag) {
-      const int row = m0 + warp * 32 + lane;
-      const bool row_ok = row < g.M;
-      const int ob = g.o_idx ? g.o_idx[b] : b;
-      const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
-      const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
-      const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
-      const long long crow = (long long)ob * g.C.bs + (long long)row * g.C.ld;
-      const long long orow = (long long)ob * g.O.bs + (long long)row * g.O.ld;
-      const long long xrow = (long long)ob * g.X.bs + (long long)row * g.X.ld;
-      float ss = 0.f;
-      int bad = 0;
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        if (n0 + c0 >= g.N) break;  // uniform across the warp
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-        if (!row_ok) continue;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = n0 + c0 + i;
-          if (col < g.N) {
-            float cval = 0.f;
-            if (need_c) {
-              cval = g.C.f32[crow + col];
-              if (g.C.lo) cval += g.C.lo[crow + col];
-            }
-            const float diag = (row == col) ? 1.f : 0.f;
-            const float r0 = g.alpha * v[i] + g.beta * cval + g.gamma * diag;
-            const float r = r0 * mult;
-            write_out(g.O, orow + col, r);
-            ss += r * r;
-            bad |= !isfinite(r);
-            if (has_x) write_out(g.X, xrow + col, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
-          }
-        }
-      }
-      if (g.sumsq) {
-#pragma unroll
-        for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) atomicAdd(g.sumsq + ob, ss);
-      }
-      if (g.status && bad) atomicOr(g.status + ob, 1);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 4) {
-    tc_fence_after();
-    tmem_dealloc(tmem, BN);
-  }
-}
-
-// ---- FP32 (3 x TF32) persistent kernel with drained accumulation ----------
-//
-// The tensor core's FP32 accumulation error grows with the number of
-// products chained into one accumulator.  Here each K-block (32 deep, 12
-// MMAs: lo*hi, hi*lo, hi*hi over 4 slices) goes into its own slot of a
-// 4-deep TMEM ring; accumulator warps drain every slot into fp32 registers
-// (round to nearest) and release it.  Two accumulator warpgroups take
-// alternate tiles, so one runs a tile's epilogue while the other drains the
-// next tile.  One CTA per SM walks the tiles of all matrices (persistent).
-//   warps 0-7  accumulator warpgroups (warp w reads TMEM lanes 32*(w%4)..)
-//   warp 8     TMEM allocator + single-thread MMA issuer
-//   warp 9     single-thread TMA producer
-
-template <int BN>
-struct Cfg3 {
-  static constexpr int A_TILE = 128 * 128;
-  static constexpr int B_TILE = BN * 128;
-  static constexpr int STAGE_BYTES = 2 * (A_TILE + B_TILE);  // hi and lo planes
-  static constexpr int STAGES_RAW = (227 * 1024 - 4096) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 6 ? 6 : STAGES_RAW;
-  static constexpr int NBUF = 4;
-  static constexpr int TCOLS = NBUF * BN;
-  static constexpr int THREADS = 320;
-  static constexpr int STAGE_OUT = 8 * 32 * 32 * 4;  // 32x32 transpose buffer per draining warp
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512 + STAGE_OUT;
-  static_assert(STAGES >= 2 && TCOLS <= 512, "FP32 tile does not fit");
-  static_assert(SMEM_BYTES <= 227 * 1024, "FP32 tile does not fit");
+struct Tile {
+  int grp, b, m0, n0, nk;
 };
+
+__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN, int BKE) {
+  Tile x;
+  x.grp = t >= p.tiles0 ? 1 : 0;
+  int r = x.grp ? t - p.tiles0 : t;
+  const int per = p.mt[x.grp] * p.nt[x.grp];
+  x.b = r / per;
+  r -= x.b * per;
+  const int mi = r / p.nt[x.grp];
+  x.m0 = mi * 128;
+  x.n0 = (r - mi * p.nt[x.grp]) * BN;
+  x.nk = (p.g[x.grp].K + BKE - 1) / BKE;
+  return x;
+}
 
 // Epilogue of a 32-row x 32-column block whose accumulators sit transposed
 // in `stage` (element (r, c) at r*32 + (c ^ r)): lane = column, so every
@@ -349,79 +166,33 @@ __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row
   }
 }
 
-struct Tile {
-  int grp, b, m0, n0, nk;
-};
-
-__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN) {
-  Tile x;
-  x.grp = t >= p.tiles0 ? 1 : 0;
-  int r = x.grp ? t - p.tiles0 : t;
-  const int per = p.mt[x.grp] * p.nt[x.grp];
-  x.b = r / per;
-  r -= x.b * per;
-  const int mi = r / p.nt[x.grp];
-  x.m0 = mi * 128;
-  x.n0 = (r - mi * p.nt[x.grp]) * BN;
-  x.nk = (p.g[x.grp].K + 31) / 32;
-  return x;
+template <int KIND>
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (KIND == 0)
+    mma_tf32(d, a, b, idesc, acc);
+  else
+    mma_f16(d, a, b, idesc, acc);
 }
 
-// Fused epilogue of one accumulator row held in registers; returns sum r^2.
-template <int BN>
-__device__ __forceinline__ float epilogue_row(const GroupDev& g, int b, int row, int n0, const float (&acc)[BN],
-                                              int& bad) {
-  if (row >= g.M) return 0.f;
-  const int ob = g.o_idx ? g.o_idx[b] : b;
-  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
-  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
-  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
-  const long long crow = (long long)ob * g.C.bs + (long long)row * g.C.ld;
-  const long long orow = (long long)ob * g.O.bs + (long long)row * g.O.ld;
-  const long long xrow = (long long)ob * g.X.bs + (long long)row * g.X.ld;
-  float ss = 0.f;
-#pragma unroll
-  for (int c = 0; c < BN; c += 16) {
-    if (n0 + c < g.N) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int col = n0 + c + i;
-        if (col < g.N) {
-          float cval = 0.f;
-          if (need_c) {
-            cval = g.C.f32[crow + col];
-            if (g.C.lo) cval += g.C.lo[crow + col];
-          }
-          const float diag = (row == col) ? 1.f : 0.f;
-          const float r0 = g.alpha * acc[c + i] + g.beta * cval + g.gamma * diag;
-          const float r = r0 * mult;
-          write_out(g.O, orow + col, r);
-          ss += r * r;
-          bad |= !isfinite(r);
-          if (has_x) write_out(g.X, xrow + col, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
-        }
-      }
-    }
-  }
-  return ss;
-}
-
-template <int BN>
-__global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg3<BN>;
+template <int KIND, int NPASS, int BN>
+__global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<KIND, NPASS, BN>;
+  using KT = KindTraits<KIND>;
   constexpr int S = C::STAGES;
   constexpr int NB = C::NBUF;
+  constexpr int BKE = C::BKE;
+  constexpr int KS = BKE / KT::KINST;  // MMA slices per K-block (4)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3 * NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * S;
-  const uint32_t tfull0 = empty0 + 8 * S;       // [NB] slot written by the MMA
-  const uint32_t tempty0 = tfull0 + 8 * 2 * NB;  // [NB] slot drained by both groups
+  const uint32_t tfull0 = empty0 + 8 * S;   // [NB] slot written by the MMA
+  const uint32_t tempty0 = tfull0 + 8 * NB;  // [NB] slot drained by both groups
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -450,7 +221,7 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
     if (lane == 0) {
       uint32_t gs = 0;
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        const Tile x = decode_tile(p, t, BN);
+        const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
         const int ab = g.a_idx ? g.a_idx[x.b] : x.b;
         const int bb = g.b_idx ? g.b_idx[x.b] : x.b;
@@ -462,25 +233,25 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
           }
           const uint32_t fb = full0 + 8 * s;
           mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-          const int k0 = kb * 32;
+          const int k0 = kb * BKE;
           uint8_t* st = smem + s * C::STAGE_BYTES;
 #pragma unroll
-          for (int pl = 0; pl < 2; ++pl) {
+          for (int pl = 0; pl < C::NPL; ++pl) {
             const CUtensorMap* ma = &p.tmA[x.grp][pl];
             const CUtensorMap* mb = &p.tmB[x.grp][pl];
             const uint32_t sa = smem_u32(st + pl * C::A_TILE);
-            const uint32_t sb = smem_u32(st + 2 * C::A_TILE + pl * C::B_TILE);
+            const uint32_t sb = smem_u32(st + C::NPL * C::A_TILE + pl * C::B_TILE);
             if (!g.a_mn) {
               tma_load_3d(sa, ma, fb, k0, x.m0, ab);
-            } else {
+            } else {  // boxes of BKE (M) x BKE (K rows)
 #pragma unroll
-              for (int j = 0; j < 4; ++j) tma_load_3d(sa + j * 4096, ma, fb, x.m0 + j * 32, k0, ab);
+              for (int j = 0; j < 128 / BKE; ++j) tma_load_3d(sa + j * BKE * 128, ma, fb, x.m0 + j * BKE, k0, ab);
             }
             if (!g.b_mn) {
               tma_load_3d(sb, mb, fb, k0, x.n0, bb);
             } else {
 #pragma unroll
-              for (int j = 0; j < BN / 32; ++j) tma_load_3d(sb + j * 4096, mb, fb, x.n0 + j * 32, k0, bb);
+              for (int j = 0; j < BN / BKE; ++j) tma_load_3d(sb + j * BKE * 128, mb, fb, x.n0 + j * BKE, k0, bb);
             }
           }
         }
@@ -488,15 +259,18 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
     }
   } else if (warp == 8) {
     if (lane == 0) {
+      constexpr uint32_t KSTEP_K = KT::KINST * C::ESZ;  // 32 bytes along a K-major row
+      constexpr uint32_t KSTEP_MN = KT::KINST * 128;    // KINST rows of 128 bytes
+      constexpr uint32_t LBO_MN = BKE * 128;            // one TMA box along M/N
       uint32_t gs = 0, gk = 0;
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
-        const Tile x = decode_tile(p, t, BN);
+        const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
-        const uint32_t idesc = idesc_f32acc(2, 2, g.a_mn, g.b_mn, 128, BN);
-        const uint32_t a_step = g.a_mn ? 1024u : 32u, b_step = g.b_mn ? 1024u : 32u;
-        const uint32_t a_lbo = g.a_mn ? 4096u : 16u, b_lbo = g.b_mn ? 4096u : 16u;
-        const uint32_t a_sbo = g.a_mn ? 512u : 1024u, b_sbo = g.b_mn ? 512u : 1024u;
-        const uint32_t a_lay = g.a_mn ? 1u : 2u, b_lay = g.b_mn ? 1u : 2u;
+        const uint32_t idesc = idesc_f32acc(KT::FMT, KT::FMT, g.a_mn, g.b_mn, 128, BN);
+        const uint32_t a_step = g.a_mn ? KSTEP_MN : KSTEP_K, b_step = g.b_mn ? KSTEP_MN : KSTEP_K;
+        const uint32_t a_lbo = g.a_mn ? LBO_MN : 16u, b_lbo = g.b_mn ? LBO_MN : 16u;
+        const uint32_t a_sbo = g.a_mn ? KT::MN_SBO : 1024u, b_sbo = g.b_mn ? KT::MN_SBO : 1024u;
+        const uint32_t a_lay = g.a_mn ? KT::MN_LAYOUT : 2u, b_lay = g.b_mn ? KT::MN_LAYOUT : 2u;
         for (int kb = 0; kb < x.nk; ++kb, ++gs, ++gk) {
           const int s = gs % S;
           const int j = gk % NB;
@@ -507,25 +281,25 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
           }
           tc_fence_after();
           uint8_t* st = smem + s * C::STAGE_BYTES;
-          const uint32_t sa0 = smem_u32(st), sb0 = smem_u32(st + 2 * C::A_TILE);
+          const uint32_t sa0 = smem_u32(st), sb0 = smem_u32(st + C::NPL * C::A_TILE);
           const uint32_t d = tmem + (uint32_t)(j * BN);
-          // the 8 small correction products first, while the accumulator is
-          // small, then the 4 hi*hi products: only those 4 additions happen
-          // at the scale of the full partial sum
+          if constexpr (NPASS == 3) {
+            // the 8 small correction products first, while the slot is small
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
-            const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
-            const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
-            const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
-            mma_tf32(d, a_lo, b_hi, idesc, ks ? 1u : 0u);
-            mma_tf32(d, a_hi, b_lo, idesc, 1u);
+            for (int ks = 0; ks < KS; ++ks) {
+              const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
+              const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
+              const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
+              const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
+              mma<KIND>(d, a_lo, b_hi, idesc, ks ? 1u : 0u);
+              mma<KIND>(d, a_hi, b_lo, idesc, 1u);
+            }
           }
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
+          for (int ks = 0; ks < KS; ++ks) {
             const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
             const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
-            mma_tf32(d, a_hi, b_hi, idesc, 1u);
+            mma<KIND>(d, a_hi, b_hi, idesc, (NPASS == 3 || ks) ? 1u : 0u);
           }
           tc_commit(empty0 + 8 * s);
           tc_commit(tfull0 + 8 * j);
@@ -533,15 +307,13 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
       }
     }
   } else {
-    // both warpgroups drain every K-block; group h owns columns
-    // [h*BN/2, (h+1)*BN/2) of the tile, warp w%4 owns TMEM lanes 32*(w%4)..
     constexpr int HC = BN / 2;
     const int h = warp >> 2;
     const int q = warp & 3;
     uint32_t gk = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
-      const Tile x = decode_tile(p, t, BN);
+      const Tile x = decode_tile(p, t, BN, BKE);
       float acc[HC];
 #pragma unroll
       for (int i = 0; i < HC; ++i) acc[i] = 0.f;
@@ -594,6 +366,8 @@ __global__ void __launch_bounds__(320, 1) gemm3_kernel(const __grid_constant__ G
   }
 }
 
+// ---- host side -------------------------------------------------------------
+
 int num_sms() {
   static int sms[64] = {0};
   int dev = 0;
@@ -606,24 +380,6 @@ int num_sms() {
   }
   return sms[dev];
 }
-
-template <int BN>
-cudaError_t run3(GemmParams& prm, cudaStream_t stream) {
-  using C = Cfg3<BN>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm3_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
-  const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
-  gemm3_kernel<BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(prm);
-  count_launch();
-  return cudaGetLastError();
-}
-
-// ---- host side -------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -654,13 +410,12 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esz,
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 template <int KIND, int NPASS, int BN>
-cudaError_t run(GemmParams& prm, int ngroups, int batch, int maxM, int maxN, cudaStream_t stream) {
+cudaError_t run(GemmParams& prm, cudaStream_t stream) {
   using C = Cfg<KIND, NPASS, BN>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -669,8 +424,8 @@ cudaError_t run(GemmParams& prm, int ngroups, int batch, int maxM, int maxN, cud
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  dim3 grid((maxN + BN - 1) / BN, (maxM + 127) / 128, ngroups * batch);
-  gemm_kernel<KIND, NPASS, BN><<<grid, 192, C::SMEM_BYTES, stream>>>(prm);
+  const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
+  gemm_kernel<KIND, NPASS, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(prm);
   count_launch();
   return cudaGetLastError();
 }
@@ -678,7 +433,7 @@ cudaError_t run(GemmParams& prm, int ngroups, int batch, int maxM, int maxN, cud
 }  // namespace
 
 cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec prec, cudaStream_t stream) {
-  if (ngroups < 1 || ngroups > 2 || batch < 1 || batch > 65535) return cudaErrorInvalidValue;
+  if (ngroups < 1 || ngroups > 2 || batch < 1) return cudaErrorInvalidValue;
   const int kind = (prec == P_FP16) ? 1 : (prec == P_BF16) ? 2 : 0;
   const int npass = (prec == P_FP32) ? 3 : 1;
   const int esz = kind ? 2 : 4;
@@ -686,22 +441,15 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
   const CUtensorMapDataType dt = kind == 0   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                  : kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  int maxM = 0, maxN = 0, minN = 1 << 30;
-  for (int i = 0; i < ngroups; ++i) {
-    maxM = groups[i].M > maxM ? groups[i].M : maxM;
-    maxN = groups[i].N > maxN ? groups[i].N : maxN;
-    minN = groups[i].N < minN ? groups[i].N : minN;
-  }
-  // Tile width: the widest that still yields a few waves of CTAs.
-  int BN = 256;
-  if (npass == 3) BN = 128;
-  if (maxN <= 64) BN = 64;
-  else if (maxN <= 128) BN = 128;
+  int maxN = 0;
+  for (int i = 0; i < ngroups; ++i) maxN = groups[i].N > maxN ? groups[i].N : maxN;
+  const int BN = maxN <= 64 ? 64 : 128;
 
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.ngroups = ngroups;
   prm.batch = batch;
+  long long total = 0;
   for (int i = 0; i < ngroups; ++i) {
     const GemmGroup& G = groups[i];
     if (G.M < 1 || G.N < 1 || G.K < 1) return cudaErrorInvalidValue;
@@ -714,44 +462,26 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
     d.a_idx = G.a_idx;
     d.b_idx = G.b_idx;
     prm.g[i] = d;
-    for (int pl = 0; pl < npass / 2 + 1 && pl < 2; ++pl) {
+    for (int pl = 0; pl < (npass == 3 ? 2 : 1); ++pl) {
       const void* abase = kind ? G.A->h16 : (pl ? (const void*)G.A->lo : (const void*)G.A->f32);
       const void* bbase = kind ? G.B->h16 : (pl ? (const void*)G.B->lo : (const void*)G.B->f32);
-      const int abx = bke, aby = G.a_mn ? bke : 128;
-      const int bbx = bke, bby = G.b_mn ? bke : BN;
-      if (!make_map(&prm.tmA[i][pl], abase, dt, esz, *G.A, abx, aby, kind == 0 && G.a_mn))
+      if (!make_map(&prm.tmA[i][pl], abase, dt, esz, *G.A, bke, G.a_mn ? bke : 128, kind == 0 && G.a_mn))
         return cudaErrorInvalidValue;
-      if (!make_map(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bbx, bby, kind == 0 && G.b_mn))
+      if (!make_map(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bke, G.b_mn ? bke : BN, kind == 0 && G.b_mn))
         return cudaErrorInvalidValue;
     }
+    prm.mt[i] = (G.M + 127) / 128;
+    prm.nt[i] = (G.N + BN - 1) / BN;
+    const long long ti = (long long)batch * prm.mt[i] * prm.nt[i];
+    if (i == 0) prm.tiles0 = (int)ti;
+    total += ti;
   }
-  if (kind == 0 && npass == 3) {  // persistent kernel over all tiles of all matrices
-    long long total = 0;
-    for (int i = 0; i < ngroups; ++i) {
-      prm.mt[i] = (groups[i].M + 127) / 128;
-      prm.nt[i] = (groups[i].N + BN - 1) / BN;
-      const long long ti = (long long)batch * prm.mt[i] * prm.nt[i];
-      if (i == 0) prm.tiles0 = (int)ti;
-      total += ti;
-    }
-    if (total > (1ll << 30)) return cudaErrorInvalidValue;
-    prm.total_tiles = (int)total;
-    if (BN == 64) return run3<64>(prm, stream);
-    return run3<128>(prm, stream);
-  }
-  if (kind == 0) {
-    if (BN == 64) return run<0, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
-    if (BN == 128) return run<0, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
-    return run<0, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
-  }
-  if (kind == 1) {
-    if (BN == 64) return run<1, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
-    if (BN == 128) return run<1, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
-    return run<1, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
-  }
-  if (BN == 64) return run<2, 1, 64>(prm, ngroups, batch, maxM, maxN, stream);
-  if (BN == 128) return run<2, 1, 128>(prm, ngroups, batch, maxM, maxN, stream);
-  return run<2, 1, 256>(prm, ngroups, batch, maxM, maxN, stream);
+  if (total > (1ll << 30)) return cudaErrorInvalidValue;
+  prm.total_tiles = (int)total;
+  if (kind == 0 && npass == 3) return BN == 64 ? run<0, 3, 64>(prm, stream) : run<0, 3, 128>(prm, stream);
+  if (kind == 0) return BN == 64 ? run<0, 1, 64>(prm, stream) : run<0, 1, 128>(prm, stream);
+  if (kind == 1) return BN == 64 ? run<1, 1, 64>(prm, stream) : run<1, 1, 128>(prm, stream);
+  return BN == 64 ? run<2, 1, 64>(prm, stream) : run<2, 1, 128>(prm, stream);
 }
 
 }  // namespace shp

@@ -89,6 +89,10 @@ struct Cfg {
   static constexpr int B_TILE = BN * 128;
   static constexpr int STAGE_BYTES = NPL * (A_TILE + B_TILE);
   static constexpr int NBUF = 4;
+  // K-blocks accumulated in one TMEM slot before it is drained: every
+  // K-block in FP32 mode (accuracy), four in the one-pass modes, whose
+  // operand rounding (2^-11) dwarfs the accumulation error
+  static constexpr int DRAIN = (NPASS == 3) ? 1 : 4;
   static constexpr int TCOLS = NBUF * BN;
   static constexpr int THREADS = 320;
   static constexpr int STAGE_OUT = 8 * 32 * 32 * 4;  // 32x32 transpose buffer per draining warp
@@ -104,17 +108,6 @@ __device__ __forceinline__ void store_h16(void* base, long long off, float v, in
     reinterpret_cast<__nv_bfloat16*>(base)[off] = __float2bfloat16_rn(v);
   else
     reinterpret_cast<__half*>(base)[off] = __float2half_rn(v);
-}
-
-__device__ __forceinline__ void write_out(const EpiOut& o, long long off, float r) {
-  if (o.lo) {
-    const float hi = tf32_round(r);
-    o.f32[off] = hi;
-    o.lo[off] = r - hi;
-  } else if (o.f32) {
-    o.f32[off] = r;
-  }
-  if (o.h16) store_h16(o.h16, off, r, o.h16_bf);
 }
 
 struct Tile {
@@ -135,34 +128,92 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN, 
   return x;
 }
 
+// One output plane set with its pointers already offset to (row0, col).
+struct OutPtrs {
+  float* f32;
+  float* lo;
+  void* h16;
+  int bf;
+  int ld;
+};
+
+__device__ __forceinline__ OutPtrs out_ptrs(const EpiOut& o, int ob, int row0, int col) {
+  OutPtrs r;
+  const long long off = (long long)ob * o.bs + (long long)row0 * o.ld + col;
+  r.f32 = o.f32 ? o.f32 + off : nullptr;
+  r.lo = o.lo ? o.lo + off : nullptr;
+  r.h16 = o.h16 ? (o.h16_bf ? (void*)(reinterpret_cast<__nv_bfloat16*>(o.h16) + off)
+                            : (void*)(reinterpret_cast<__half*>(o.h16) + off))
+                : nullptr;
+  r.bf = o.h16_bf;
+  r.ld = o.ld;
+  return r;
+}
+
+__device__ __forceinline__ void put(const OutPtrs& o, int r, float v) {
+  const long long off = (long long)r * o.ld;
+  if (o.lo) {
+    const float hi = tf32_round(v);
+    o.f32[off] = hi;
+    o.lo[off] = v - hi;
+  } else if (o.f32) {
+    o.f32[off] = v;
+  }
+  if (o.h16) store_h16(o.h16, off, v, o.bf);
+}
+
 // Epilogue of a 32-row x 32-column block whose accumulators sit transposed
 // in `stage` (element (r, c) at r*32 + (c ^ r)): lane = column, so every
 // load of C and every store of an output plane is one 128-byte segment.
+// Rows go in groups of 8 so that loads and stores of a group overlap.
 __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row0, int col, const float* stage,
                                                int lane, float& ss, int& bad) {
+  if (col >= g.N) return;
   const int ob = g.o_idx ? g.o_idx[b] : b;
   const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
   const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
   const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
-  if (col >= g.N) return;
-  long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
-  long long ooff = (long long)ob * g.O.bs + (long long)row0 * g.O.ld + col;
-  long long xoff = (long long)ob * g.X.bs + (long long)row0 * g.X.ld + col;
+  const OutPtrs O = out_ptrs(g.O, ob, row0, col);
+  const OutPtrs X = has_x ? out_ptrs(g.X, ob, row0, col) : O;
+  const float* cf = nullptr;
+  const float* cl = nullptr;
+  int cld = 0;
+  if (need_c) {
+    const long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
+    cf = g.C.f32 + coff;
+    cl = g.C.lo ? g.C.lo + coff : nullptr;
+    cld = g.C.ld;
+  }
+  const float alpha = g.alpha, beta = g.beta, gamma = g.gamma;
+  const float alpha2 = g.alpha2, beta2 = g.beta2, gamma2 = g.gamma2;
   const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
-  for (int r = 0; r < rmax; ++r, coff += g.C.ld, ooff += g.O.ld, xoff += g.X.ld) {
-    const float a = stage[r * 32 + (lane ^ r)];
-    float cval = 0.f;
-    if (need_c) {
-      cval = g.C.f32[coff];
-      if (g.C.lo) cval += g.C.lo[coff];
+  const int dr = col - row0;  // the diagonal sits in row dr of this block
+#pragma unroll 1
+  for (int r0 = 0; r0 < rmax; r0 += 8) {
+    float a[8], cv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + i;
+      a[i] = stage[r * 32 + (lane ^ r)];
+      cv[i] = 0.f;
+      if (need_c && r < rmax) {
+        cv[i] = cf[(long long)r * cld];
+        if (cl) cv[i] += cl[(long long)r * cld];
+      }
     }
-    const float diag = (row0 + r == col) ? 1.f : 0.f;
-    const float r0 = g.alpha * a + g.beta * cval + g.gamma * diag;
-    const float v = r0 * mult;
-    write_out(g.O, ooff, v);
-    ss += v * v;
-    bad |= !isfinite(v);
-    if (has_x) write_out(g.X, xoff, mult * (g.alpha2 * r0 + g.beta2 * cval + g.gamma2 * diag));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = r0 + i;
+      if (r < rmax) {
+        const float diag = (r == dr) ? 1.f : 0.f;
+        const float q0 = alpha * a[i] + beta * cv[i] + gamma * diag;
+        const float v = q0 * mult;
+        put(O, r, v);
+        ss += v * v;
+        bad |= !isfinite(v);
+        if (has_x) put(X, r, mult * (alpha2 * q0 + beta2 * cv[i] + gamma2 * diag));
+      }
+    }
   }
 }
 
@@ -174,6 +225,18 @@ __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t
     mma_f16(d, a, b, idesc, acc);
 }
 
+// Ring position: index and the parity of its current round.
+struct Ring {
+  uint32_t i = 0, ph = 0;
+  template <int N>
+  __device__ __forceinline__ void next() {
+    if (++i == N) {
+      i = 0;
+      ph ^= 1;
+    }
+  }
+};
+
 template <int KIND, int NPASS, int BN>
 __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<KIND, NPASS, BN>;
@@ -181,18 +244,20 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
   constexpr int S = C::STAGES;
   constexpr int NB = C::NBUF;
   constexpr int BKE = C::BKE;
+  constexpr int DR = C::DRAIN;
   constexpr int KS = BKE / KT::KINST;  // MMA slices per K-block (4)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * S;
-  const uint32_t tfull0 = empty0 + 8 * S;   // [NB] slot written by the MMA
-  const uint32_t tempty0 = tfull0 + 8 * NB;  // [NB] slot drained by both groups
+  const uint32_t tfull0 = empty0 + 8 * S;    // [NB] slot written by the MMA
+  const uint32_t tempty0 = tfull0 + 8 * NB;  // [NB] slot drained by all 8 draining warps
+  const uint32_t done_bar = tempty0 + 8 * NB;  // last MMAs of this CTA complete
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -201,8 +266,9 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
     }
     for (int j = 0; j < NB; ++j) {
       mbar_init(tfull0 + 8 * j, 1);
-      mbar_init(tempty0 + 8 * j, 256);  // every thread of both draining warpgroups
+      mbar_init(tempty0 + 8 * j, 8);  // one arrival per draining warp
     }
+    mbar_init(done_bar, 1);
     // skip all tiles once any CTA has given up on a barrier
     *abort_flag = (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) ? 1 : 0;
     fence_barrier_init();
@@ -218,99 +284,128 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
   const int total = p.total_tiles;
 
   if (warp == 9) {
+    // ---- TMA producer ----
     if (lane == 0) {
-      uint32_t gs = 0;
+      Ring st;
+      long long issued = 0;
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
         const int ab = g.a_idx ? g.a_idx[x.b] : x.b;
         const int bb = g.b_idx ? g.b_idx[x.b] : x.b;
-        for (int kb = 0; kb < x.nk; ++kb, ++gs) {
-          const int s = gs % S;
-          if (gs >= S && !mbar_wait(empty0 + 8 * s, ((gs / S) - 1) & 1)) {
-            *abort_flag = 1;
+        const CUtensorMap* ma = &p.tmA[x.grp][0];
+        const CUtensorMap* mb = &p.tmB[x.grp][0];
+        const int a_mn = g.a_mn, b_mn = g.b_mn;
+        bool ok = true;
+        for (int kb = 0, k0 = 0; kb < x.nk; ++kb, k0 += BKE) {
+          if (!mbar_wait(empty0 + 8 * st.i, st.ph ^ 1)) {
+            ok = false;
             break;
           }
-          const uint32_t fb = full0 + 8 * s;
+          const uint32_t fb = full0 + 8 * st.i;
           mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-          const int k0 = kb * BKE;
-          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const uint32_t sa = smem_u32(smem + st.i * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::NPL * C::A_TILE;
 #pragma unroll
           for (int pl = 0; pl < C::NPL; ++pl) {
-            const CUtensorMap* ma = &p.tmA[x.grp][pl];
-            const CUtensorMap* mb = &p.tmB[x.grp][pl];
-            const uint32_t sa = smem_u32(st + pl * C::A_TILE);
-            const uint32_t sb = smem_u32(st + C::NPL * C::A_TILE + pl * C::B_TILE);
-            if (!g.a_mn) {
-              tma_load_3d(sa, ma, fb, k0, x.m0, ab);
+            if (!a_mn) {
+              tma_load_3d(sa + pl * C::A_TILE, ma + pl, fb, k0, x.m0, ab);
             } else {  // boxes of BKE (M) x BKE (K rows)
 #pragma unroll
-              for (int j = 0; j < 128 / BKE; ++j) tma_load_3d(sa + j * BKE * 128, ma, fb, x.m0 + j * BKE, k0, ab);
+              for (int j = 0; j < 128 / BKE; ++j)
+                tma_load_3d(sa + pl * C::A_TILE + j * BKE * 128, ma + pl, fb, x.m0 + j * BKE, k0, ab);
             }
-            if (!g.b_mn) {
-              tma_load_3d(sb, mb, fb, k0, x.n0, bb);
+            if (!b_mn) {
+              tma_load_3d(sb + pl * C::B_TILE, mb + pl, fb, k0, x.n0, bb);
             } else {
 #pragma unroll
-              for (int j = 0; j < BN / BKE; ++j) tma_load_3d(sb + j * BKE * 128, mb, fb, x.n0 + j * BKE, k0, bb);
+              for (int j = 0; j < BN / BKE; ++j)
+                tma_load_3d(sb + pl * C::B_TILE + j * BKE * 128, mb + pl, fb, x.n0 + j * BKE, k0, bb);
             }
           }
+          st.template next<S>();
+          ++issued;
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
         }
       }
+      // after an abort, loads may still be landing in stages nobody waited
+      // for: let the latest load of every stage finish before the shared
+      // memory is given up (immediate when all were consumed)
+      for (long long n = issued - 1; n >= 0 && n >= issued - S; --n) mbar_wait(full0 + 8 * (n % S), (n / S) & 1);
     }
   } else if (warp == 8) {
+    // ---- MMA issuer ----
     if (lane == 0) {
       constexpr uint32_t KSTEP_K = KT::KINST * C::ESZ;  // 32 bytes along a K-major row
       constexpr uint32_t KSTEP_MN = KT::KINST * 128;    // KINST rows of 128 bytes
       constexpr uint32_t LBO_MN = BKE * 128;            // one TMA box along M/N
-      uint32_t gs = 0, gk = 0;
+      const uint32_t smem0 = smem_u32(smem);
+      Ring st, sl;
+      int in_slot = 0;  // K-blocks already accumulated in the current slot
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
         const uint32_t idesc = idesc_f32acc(KT::FMT, KT::FMT, g.a_mn, g.b_mn, 128, BN);
-        const uint32_t a_step = g.a_mn ? KSTEP_MN : KSTEP_K, b_step = g.b_mn ? KSTEP_MN : KSTEP_K;
-        const uint32_t a_lbo = g.a_mn ? LBO_MN : 16u, b_lbo = g.b_mn ? LBO_MN : 16u;
-        const uint32_t a_sbo = g.a_mn ? KT::MN_SBO : 1024u, b_sbo = g.b_mn ? KT::MN_SBO : 1024u;
-        const uint32_t a_lay = g.a_mn ? KT::MN_LAYOUT : 2u, b_lay = g.b_mn ? KT::MN_LAYOUT : 2u;
-        for (int kb = 0; kb < x.nk; ++kb, ++gs, ++gk) {
-          const int s = gs % S;
-          const int j = gk % NB;
-          if (!mbar_wait(full0 + 8 * s, (gs / S) & 1) ||
-              (gk >= NB && !mbar_wait(tempty0 + 8 * j, ((gk / NB) - 1) & 1))) {
-            *abort_flag = 1;
+        // descriptors of stage 0; the start-address field (address >> 4)
+        // never carries out of its 14 bits inside shared memory, so the
+        // stage and slice offsets are added to the 64-bit descriptor
+        const uint64_t a0 = g.a_mn ? sdesc_sw128(smem0, LBO_MN, KT::MN_SBO, KT::MN_LAYOUT)
+                                   : sdesc_sw128(smem0, 16u, 1024u, 2u);
+        const uint64_t b0 = g.b_mn ? sdesc_sw128(smem0 + C::NPL * C::A_TILE, LBO_MN, KT::MN_SBO, KT::MN_LAYOUT)
+                                   : sdesc_sw128(smem0 + C::NPL * C::A_TILE, 16u, 1024u, 2u);
+        const uint64_t a_step = (g.a_mn ? KSTEP_MN : KSTEP_K) >> 4;
+        const uint64_t b_step = (g.b_mn ? KSTEP_MN : KSTEP_K) >> 4;
+        bool ok = true;
+        for (int kb = 0; kb < x.nk; ++kb) {
+          if (!mbar_wait(full0 + 8 * st.i, st.ph) || (in_slot == 0 && !mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1))) {
+            ok = false;
             break;
           }
           tc_fence_after();
-          uint8_t* st = smem + s * C::STAGE_BYTES;
-          const uint32_t sa0 = smem_u32(st), sb0 = smem_u32(st + C::NPL * C::A_TILE);
-          const uint32_t d = tmem + (uint32_t)(j * BN);
+          const uint64_t so = (uint64_t)(st.i * (C::STAGE_BYTES >> 4));
+          const uint64_t ad = a0 + so, bd = b0 + so;
+          const uint32_t d = tmem + sl.i * BN;
           if constexpr (NPASS == 3) {
             // the 8 small correction products first, while the slot is small
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-              const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
-              const uint64_t a_lo = sdesc_sw128(sa0 + C::A_TILE + ks * a_step, a_lbo, a_sbo, a_lay);
-              const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
-              const uint64_t b_lo = sdesc_sw128(sb0 + C::B_TILE + ks * b_step, b_lbo, b_sbo, b_lay);
-              mma<KIND>(d, a_lo, b_hi, idesc, ks ? 1u : 0u);
-              mma<KIND>(d, a_hi, b_lo, idesc, 1u);
+              mma<KIND>(d, ad + (C::A_TILE >> 4) + ks * a_step, bd + ks * b_step, idesc, ks ? 1u : 0u);
+              mma<KIND>(d, ad + ks * a_step, bd + (C::B_TILE >> 4) + ks * b_step, idesc, 1u);
             }
-          }
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            const uint64_t a_hi = sdesc_sw128(sa0 + ks * a_step, a_lbo, a_sbo, a_lay);
-            const uint64_t b_hi = sdesc_sw128(sb0 + ks * b_step, b_lbo, b_sbo, b_lay);
-            mma<KIND>(d, a_hi, b_hi, idesc, (NPASS == 3 || ks) ? 1u : 0u);
+            for (int ks = 0; ks < KS; ++ks) mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, 1u);
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks)
+              mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, (in_slot | ks) ? 1u : 0u);
           }
-          tc_commit(empty0 + 8 * s);
-          tc_commit(tfull0 + 8 * j);
+          tc_commit(empty0 + 8 * st.i);
+          st.template next<S>();
+          if (++in_slot == DR || kb == x.nk - 1) {
+            tc_commit(tfull0 + 8 * sl.i);
+            sl.template next<NB>();
+            in_slot = 0;
+          }
+        }
+        if (!ok) {
+          *abort_flag = 1;
+          break;
         }
       }
+      // every MMA of this CTA has finished before TMEM is given up
+      tc_commit(done_bar);
+      mbar_wait(done_bar, 0);
     }
   } else {
+    // ---- draining warps + epilogue ----
     constexpr int HC = BN / 2;
     const int h = warp >> 2;
     const int q = warp & 3;
-    uint32_t gk = 0;
+    Ring sl;
+    float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + warp * 1024;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
       const Tile x = decode_tile(p, t, BN, BKE);
@@ -318,29 +413,30 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
 #pragma unroll
       for (int i = 0; i < HC; ++i) acc[i] = 0.f;
       bool ok = true;
-      for (int kb = 0; kb < x.nk; ++kb, ++gk) {
-        const int j = gk % NB;
-        ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * j, (gk / NB) & 1));
+      const int nslots = (x.nk + DR - 1) / DR;
+      for (int u = 0; u < nslots; ++u) {
+        ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * sl.i, sl.ph));
         if (!ok) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
         uint32_t r[HC];
-        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(j * BN + h * HC);
+        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(sl.i * BN + h * HC);
 #pragma unroll
         for (int c = 0; c < HC; c += 32) tmem_ld32_nowait(base + c, r + c);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < HC; ++i) acc[i] += __uint_as_float(r[i]);
         tc_fence_before();
-        mbar_arrive(tempty0 + 8 * j);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty0 + 8 * sl.i);
+        sl.template next<NB>();
       }
       if (!ok) break;
       const GroupDev& g = p.g[x.grp];
       int bad = 0;
       float ss = 0.f;
-      float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + warp * 1024;
 #pragma unroll
       for (int ch = 0; ch < HC / 32; ++ch) {
 #pragma unroll

@@ -150,22 +150,42 @@ __device__ __forceinline__ OutPtrs out_ptrs(const EpiOut& o, int ob, int row0, i
   return r;
 }
 
-__device__ __forceinline__ void put(const OutPtrs& o, int r, float v) {
-  const long long off = (long long)r * o.ld;
+// Stores rows [r0, r0 + 8) of values v (rows >= rmax skipped) into one
+// output plane set; the format tests are uniform and sit outside the rows.
+__device__ __forceinline__ void put_rows(const OutPtrs& o, int r0, int rmax, const float (&v)[8]) {
+  const long long ld = o.ld;
   if (o.lo) {
-    const float hi = tf32_round(v);
-    o.f32[off] = hi;
-    o.lo[off] = v - hi;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (r0 + i < rmax) {
+        const float hi = tf32_round(v[i]);
+        o.f32[(r0 + i) * ld] = hi;
+        o.lo[(r0 + i) * ld] = v[i] - hi;
+      }
   } else if (o.f32) {
-    o.f32[off] = v;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (r0 + i < rmax) o.f32[(r0 + i) * ld] = v[i];
   }
-  if (o.h16) store_h16(o.h16, off, v, o.bf);
+  if (o.h16) {
+    if (o.bf) {
+      __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(o.h16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (r0 + i < rmax) h[(r0 + i) * ld] = __float2bfloat16_rn(v[i]);
+    } else {
+      __half* h = reinterpret_cast<__half*>(o.h16);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (r0 + i < rmax) h[(r0 + i) * ld] = __float2half_rn(v[i]);
+    }
+  }
 }
 
 // Epilogue of a 32-row x 32-column block whose accumulators sit transposed
 // in `stage` (element (r, c) at r*32 + (c ^ r)): lane = column, so every
 // load of C and every store of an output plane is one 128-byte segment.
-// Rows go in groups of 8 so that loads and stores of a group overlap.
+// Rows go in groups of 8: values first, then the stores of the group.
 __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row0, int col, const float* stage,
                                                int lane, float& ss, int& bad) {
   if (col >= g.N) return;
@@ -177,7 +197,7 @@ __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row
   const OutPtrs X = has_x ? out_ptrs(g.X, ob, row0, col) : O;
   const float* cf = nullptr;
   const float* cl = nullptr;
-  int cld = 0;
+  long long cld = 0;
   if (need_c) {
     const long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
     cf = g.C.f32 + coff;
@@ -190,29 +210,122 @@ __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row
   const int dr = col - row0;  // the diagonal sits in row dr of this block
 #pragma unroll 1
   for (int r0 = 0; r0 < rmax; r0 += 8) {
-    float a[8], cv[8];
+    float cv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cv[i] = 0.f;
+    if (need_c) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (r0 + i < rmax) cv[i] = cf[(r0 + i) * cld] + (cl ? cl[(r0 + i) * cld] : 0.f);
+    }
+    float v[8], xv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = r0 + i;
-      a[i] = stage[r * 32 + (lane ^ r)];
-      cv[i] = 0.f;
-      if (need_c && r < rmax) {
-        cv[i] = cf[(long long)r * cld];
-        if (cl) cv[i] += cl[(long long)r * cld];
+      const float diag = (r == dr) ? 1.f : 0.f;
+      const float q0 = alpha * stage[r * 32 + (lane ^ r)] + beta * cv[i] + gamma * diag;
+      v[i] = q0 * mult;
+      xv[i] = mult * (alpha2 * q0 + beta2 * cv[i] + gamma2 * diag);
+      if (r < rmax) {
+        ss += v[i] * v[i];
+        bad |= !isfinite(v[i]);
       }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + i;
-      if (r < rmax) {
-        const float diag = (r == dr) ? 1.f : 0.f;
-        const float q0 = alpha * a[i] + beta * cv[i] + gamma * diag;
-        const float v = q0 * mult;
-        put(O, r, v);
-        ss += v * v;
-        bad |= !isfinite(v);
-        if (has_x) put(X, r, mult * (alpha2 * q0 + beta2 * cv[i] + gamma2 * diag));
+    put_rows(O, r0, rmax, v);
+    if (has_x) put_rows(X, r0, rmax, xv);
+  }
+}
+
+// 16-byte version of the epilogue for one 32x32 block: the block sits in
+// `stage` as rows of eight float4 slots, slot j of row r at r*8 + (j ^ (r&7));
+// each lane handles four consecutive columns of one row, a warp four rows
+// per step, so each store is a 128-byte row segment per eight lanes.
+__device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) {
+  if (o.lo) {
+    float4 hi;
+    hi.x = tf32_round(v.x);
+    hi.y = tf32_round(v.y);
+    hi.z = tf32_round(v.z);
+    hi.w = tf32_round(v.w);
+    *reinterpret_cast<float4*>(o.f32 + off) = hi;
+    *reinterpret_cast<float4*>(o.lo + off) = make_float4(v.x - hi.x, v.y - hi.y, v.z - hi.z, v.w - hi.w);
+  } else if (o.f32) {
+    *reinterpret_cast<float4*>(o.f32 + off) = v;
+  }
+  if (o.h16) {
+    if (o.bf) {
+      __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&a);
+      u.y = *reinterpret_cast<uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(o.h16) + off) = u;
+    } else {
+      __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&a);
+      u.y = *reinterpret_cast<uint32_t*>(&b);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) = u;
+    }
+  }
+}
+
+__device__ __forceinline__ void epilogue_block4(const GroupDev& g, int b, int row0, int col0, const float4* stage,
+                                                int lane, float& ss, int& bad) {
+  const int cq = lane & 7;
+  const int col = col0 + 4 * cq;
+  if (col >= g.N) return;
+  const int ob = g.o_idx ? g.o_idx[b] : b;
+  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
+  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
+  const OutPtrs O = out_ptrs(g.O, ob, row0, col);
+  const OutPtrs X = has_x ? out_ptrs(g.X, ob, row0, col) : O;
+  const float* cf = nullptr;
+  const float* cl = nullptr;
+  long long cld = 0;
+  if (need_c) {
+    const long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
+    cf = g.C.f32 + coff;
+    cl = g.C.lo ? g.C.lo + coff : nullptr;
+    cld = g.C.ld;
+  }
+  const float alpha = g.alpha, beta = g.beta, gamma = g.gamma;
+  const float alpha2 = g.alpha2, beta2 = g.beta2, gamma2 = g.gamma2;
+  const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
+    const int r = it * 4 + (lane >> 3);
+    if (r >= rmax) continue;
+    const float4 a = stage[r * 8 + (cq ^ (r & 7))];
+    float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (need_c) {
+      c = *reinterpret_cast<const float4*>(cf + r * cld);
+      if (cl) {
+        const float4 l = *reinterpret_cast<const float4*>(cl + r * cld);
+        c.x += l.x;
+        c.y += l.y;
+        c.z += l.z;
+        c.w += l.w;
       }
+    }
+    const int e = row0 + r - col;  // component on the diagonal, if 0..3
+    const float d0 = e == 0 ? 1.f : 0.f, d1 = e == 1 ? 1.f : 0.f, d2 = e == 2 ? 1.f : 0.f, d3 = e == 3 ? 1.f : 0.f;
+    float4 q;
+    q.x = alpha * a.x + beta * c.x + gamma * d0;
+    q.y = alpha * a.y + beta * c.y + gamma * d1;
+    q.z = alpha * a.z + beta * c.z + gamma * d2;
+    q.w = alpha * a.w + beta * c.w + gamma * d3;
+    const float4 v = make_float4(q.x * mult, q.y * mult, q.z * mult, q.w * mult);
+    const long long off = (long long)r * O.ld;
+    put4(O, off, v);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+    if (has_x) {
+      const float4 xv = make_float4(mult * (alpha2 * q.x + beta2 * c.x + gamma2 * d0),
+                                    mult * (alpha2 * q.y + beta2 * c.y + gamma2 * d1),
+                                    mult * (alpha2 * q.z + beta2 * c.z + gamma2 * d2),
+                                    mult * (alpha2 * q.w + beta2 * c.w + gamma2 * d3));
+      put4(X, (long long)r * X.ld, xv);
     }
   }
 }
@@ -296,6 +409,7 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         const CUtensorMap* ma = &p.tmA[x.grp][0];
         const CUtensorMap* mb = &p.tmB[x.grp][0];
         const int a_mn = g.a_mn, b_mn = g.b_mn;
+        const int a4 = p.a4d[x.grp], b4 = p.b4d[x.grp];
         bool ok = true;
         for (int kb = 0, k0 = 0; kb < x.nk; ++kb, k0 += BKE) {
           if (!mbar_wait(empty0 + 8 * st.i, st.ph ^ 1)) {
@@ -310,6 +424,8 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
           for (int pl = 0; pl < C::NPL; ++pl) {
             if (!a_mn) {
               tma_load_3d(sa + pl * C::A_TILE, ma + pl, fb, k0, x.m0, ab);
+            } else if (a4) {
+              tma_load_4d(sa + pl * C::A_TILE, ma + pl, fb, 0, k0, x.m0 / BKE, ab);
             } else {  // boxes of BKE (M) x BKE (K rows)
 #pragma unroll
               for (int j = 0; j < 128 / BKE; ++j)
@@ -317,6 +433,8 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
             }
             if (!b_mn) {
               tma_load_3d(sb + pl * C::B_TILE, mb + pl, fb, k0, x.n0, bb);
+            } else if (b4) {
+              tma_load_4d(sb + pl * C::B_TILE, mb + pl, fb, 0, k0, x.n0 / BKE, bb);
             } else {
 #pragma unroll
               for (int j = 0; j < BN / BKE; ++j)
@@ -437,13 +555,27 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       const GroupDev& g = p.g[x.grp];
       int bad = 0;
       float ss = 0.f;
+      if (g.vec4) {
+        float4* stage4 = reinterpret_cast<float4*>(stage);
 #pragma unroll
-      for (int ch = 0; ch < HC / 32; ++ch) {
+        for (int ch = 0; ch < HC / 32; ++ch) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = acc[ch * 32 + c];
-        __syncwarp();
-        epilogue_block(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad);
-        __syncwarp();
+          for (int j = 0; j < 8; ++j)
+            stage4[lane * 8 + (j ^ (lane & 7))] = make_float4(acc[ch * 32 + 4 * j], acc[ch * 32 + 4 * j + 1],
+                                                              acc[ch * 32 + 4 * j + 2], acc[ch * 32 + 4 * j + 3]);
+          __syncwarp();
+          epilogue_block4(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32, stage4, lane, ss, bad);
+          __syncwarp();
+        }
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < HC / 32; ++ch) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = acc[ch * 32 + c];
+          __syncwarp();
+          epilogue_block(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad);
+          __syncwarp();
+        }
       }
       if (g.sumsq) {
 #pragma unroll
@@ -510,6 +642,24 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esz,
   return r == CUDA_SUCCESS;
 }
 
+// 4-D view of an MN-major plane: {bk inner elements, rows (K), column
+// chunk, matrix}; one box = `chunks` chunks of bk x bk, stored chunk after
+// chunk (the layout of the multi-box loads).  Needs ld % bk == 0 so that
+// the last chunk of a row stays inside the padded row.
+bool make_map_4d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esz, const Planes& P, int bk,
+                 int chunks, bool atom32) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || !base) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)bk, (cuuint64_t)P.rows, (cuuint64_t)((P.cols + bk - 1) / bk), (cuuint64_t)P.count};
+  cuuint64_t strides[3] = {(cuuint64_t)P.ld * esz, (cuuint64_t)bk * esz, (cuuint64_t)P.bs * esz};
+  cuuint32_t box[4] = {(cuuint32_t)bk, (cuuint32_t)bk, (cuuint32_t)chunks, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int KIND, int NPASS, int BN>
 cudaError_t run(GemmParams& prm, cudaStream_t stream) {
   using C = Cfg<KIND, NPASS, BN>;
@@ -558,13 +708,35 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
     d.a_idx = G.a_idx;
     d.b_idx = G.b_idx;
     prm.g[i] = d;
+    prm.a4d[i] = G.a_mn && G.A->ld % bke == 0;
+    {
+      auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
+      auto al8 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 7u) == 0; };
+      auto ok_out = [&](const EpiOut& o) {
+        return (o.ld % 4 == 0) && (o.bs % 4 == 0) && al16(o.f32) && al16(o.lo) && al8(o.h16);
+      };
+      const bool has_x = d.X.f32 || d.X.h16;
+      const bool need_c = d.beta != 0.f || (has_x && d.beta2 != 0.f);
+      bool v = G.N % 4 == 0 && ok_out(d.O) && (!has_x || ok_out(d.X));
+      if (need_c) v = v && d.C.ld % 4 == 0 && d.C.bs % 4 == 0 && al16(d.C.f32) && al16(d.C.lo);
+      prm.g[i].vec4 = v ? 1 : 0;
+    }
+    prm.b4d[i] = G.b_mn && G.B->ld % bke == 0;
     for (int pl = 0; pl < (npass == 3 ? 2 : 1); ++pl) {
       const void* abase = kind ? G.A->h16 : (pl ? (const void*)G.A->lo : (const void*)G.A->f32);
       const void* bbase = kind ? G.B->h16 : (pl ? (const void*)G.B->lo : (const void*)G.B->f32);
-      if (!make_map(&prm.tmA[i][pl], abase, dt, esz, *G.A, bke, G.a_mn ? bke : 128, kind == 0 && G.a_mn))
+      if (prm.a4d[i]) {
+        if (!make_map_4d(&prm.tmA[i][pl], abase, dt, esz, *G.A, bke, 128 / bke, kind == 0))
+          return cudaErrorInvalidValue;
+      } else if (!make_map(&prm.tmA[i][pl], abase, dt, esz, *G.A, bke, G.a_mn ? bke : 128, kind == 0 && G.a_mn)) {
         return cudaErrorInvalidValue;
-      if (!make_map(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bke, G.b_mn ? bke : BN, kind == 0 && G.b_mn))
+      }
+      if (prm.b4d[i]) {
+        if (!make_map_4d(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bke, BN / bke, kind == 0))
+          return cudaErrorInvalidValue;
+      } else if (!make_map(&prm.tmB[i][pl], bbase, dt, esz, *G.B, bke, G.b_mn ? bke : BN, kind == 0 && G.b_mn)) {
         return cudaErrorInvalidValue;
+      }
     }
     prm.mt[i] = (G.M + 127) / 128;
     prm.nt[i] = (G.N + BN - 1) / BN;

@@ -61,6 +61,7 @@ struct GroupDev {
   float alpha2 = 0.f, beta2 = 0.f, gamma2 = 0.f;
   float* sumsq = nullptr;
   int* status = nullptr;
+  int vec4 = 0;  // set by the launcher: N, leading dimensions and bases allow 16-byte row segments
 };
 
 struct alignas(64) GemmParams {
@@ -73,6 +74,9 @@ struct alignas(64) GemmParams {
   // come first, then group 1
   int mt[2], nt[2];
   int tiles0, total_tiles;
+  // 1: the MN-major operand's map is a 4-D view (inner BK-element chunk,
+  // K rows, chunk index, matrix) that brings a whole tile in one load
+  int a4d[2], b4d[2];
 };
 
 // Host description of one group before tensor maps are built.

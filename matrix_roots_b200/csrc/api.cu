@@ -82,8 +82,11 @@ Planes make_planes(Carver& c, int count, int rows, int cols, Prec prec, bool nee
   P.count = count;
   const size_t n = (size_t)count * (size_t)P.bs;
   if (prec == P_FP32) {
-    P.f32 = static_cast<float*>(c.take(n * 4));
-    P.lo = static_cast<float*>(c.take(n * 4));
+    if (need_f32) P.f32 = static_cast<float*>(c.take(n * 4));
+    P.h16 = c.take(n * 2);
+    P.h16lo = c.take(n * 2);
+    P.exp = static_cast<int*>(c.take(sizeof(int) * count));
+    P.amax = static_cast<float*>(c.take(sizeof(float) * count));
   } else if (prec == P_TF32) {
     P.f32 = static_cast<float*>(c.take(n * 4));
   } else {
@@ -97,16 +100,21 @@ Planes make_planes(Carver& c, int count, int rows, int cols, Prec prec, bool nee
 EpiC as_c(const Planes& P) {
   EpiC c;
   c.f32 = P.f32;
-  c.lo = P.lo;
+  c.amax = P.amax;
   c.ld = P.ld;
   c.bs = P.bs;
   return c;
 }
-EpiOut as_out(const Planes& P) {
+// Output into planes; with full = false the fp32 copy of the FP32 / FP16 /
+// BF16 planes is not written (the value is only read by tensor-core passes).
+EpiOut as_out(const Planes& P, bool full = true) {
   EpiOut o;
-  o.f32 = P.f32;
-  o.lo = P.lo;
+  o.f32 = (full || !(P.h16)) ? P.f32 : nullptr;
   o.h16 = P.h16;
+  o.h16lo = P.h16lo;
+  o.exp = P.exp;
+  o.amax = P.amax;
+  o.amax_n = P.amax ? P.count : 0;
   o.h16_bf = P.h16_bf;
   o.ld = P.ld;
   o.bs = P.bs;
@@ -173,7 +181,8 @@ RootBufs carve_roots(Carver& c, int count, int n, int method, Prec pr, int scali
   } else {
     r.Y[0] = make_planes(c, count, n, n, pr);  // S
     r.Z[0] = make_planes(c, count, n, n, pr);  // B_{k+1}
-    r.Z[1] = make_planes(c, count, n, n, pr);  // B_{k+2} / B_k
+    r.Z[1] = make_planes(c, count, n, n, pr);  // B_{k+2}
+    r.T = make_planes(c, count, n, n, pr);     // B_k
   }
   if (scaling == SHP_SCALE_POWER) {
     r.fscale = static_cast<float*>(c.take(sizeof(float) * count));
@@ -248,12 +257,13 @@ shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec 
   int cur = 0;
   for (int call = 0; call < 2; ++call) {
     // iteration 1 (Z_0 = I): Y_1 = Y_0 (3I - Y_0)/2 = 1.5 Y_0 - 0.5 Y_0^2, Z_1 = 1.5 I - 0.5 Y_0
+    // Y keeps its fp32 copy only where it will be the next call's C
     GemmGroup g = group(n, n, n, &r.Y[cur], 0, &r.Y[cur], 1);
     g.epi.alpha = -0.5f;
     g.epi.beta = 1.5f;
     g.epi.C = as_c(r.Y[cur]);
-    g.epi.O = as_out(r.Y[1 - cur]);
-    g.epi.X = as_out(r.Z[1 - cur]);
+    g.epi.O = as_out(r.Y[1 - cur], call == 0 && iters == 1);
+    g.epi.X = as_out(r.Z[1 - cur], false);
     g.epi.beta2 = -0.5f;
     g.epi.gamma2 = 1.5f;
     if (call == 1 && iters == 1) {
@@ -269,14 +279,14 @@ shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec 
       GemmGroup gt = group(n, n, n, &r.Z[cur], 0, &r.Y[cur], 1);
       gt.epi.alpha = -0.5f;
       gt.epi.gamma = 1.5f;
-      gt.epi.O = as_out(r.T);
+      gt.epi.O = as_out(r.T, false);
       GEMM_TRY(launch_gemm(&gt, 1, count, pr, st));
       // Y' = Y T and Z' = T Z in one grouped launch (drop what is not needed)
       GemmGroup gs[2];
       int ng = 0;
       if (!(call == 1 && last)) {
         gs[ng] = group(n, n, n, &r.Y[cur], 0, &r.T, 1);
-        gs[ng].epi.O = as_out(r.Y[1 - cur]);
+        gs[ng].epi.O = as_out(r.Y[1 - cur], call == 0 && last);
         ++ng;
       }
       if (!(call == 0 && last)) {
@@ -286,7 +296,7 @@ shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec 
           gs[ng].epi.bscale = scale;
           gs[ng].epi.status = status;
         } else {
-          gs[ng].epi.O = as_out(r.Z[1 - cur]);
+          gs[ng].epi.O = as_out(r.Z[1 - cur], false);
         }
         ++ng;
       }
@@ -328,22 +338,22 @@ shp_status run_cn(const float* A, int count, int n, float eps, int iters, Prec p
         GEMM_TRY(launch_gemm(gs, 1, count, pr, st));
         break;
       }
-      gs[0].epi.O = as_out(Xp[1 - cx]);
+      gs[0].epi.O = as_out(Xp[1 - cx], false);
       gs[1] = group(n, n, n, &r.T, 0, &r.T, 1);  // T^2 = T T
-      gs[1].epi.O = as_out(r.T2);
+      gs[1].epi.O = as_out(r.T2, false);
       GEMM_TRY(launch_gemm(gs, 2, count, pr, st));
       cx = 1 - cx;
     } else {
       GemmGroup g2 = group(n, n, n, &r.T, 0, &r.T, 1);  // T_0^2
-      g2.epi.O = as_out(r.T2);
+      g2.epi.O = as_out(r.T2, false);
       GEMM_TRY(launch_gemm(&g2, 1, count, pr, st));
     }
     GemmGroup g4 = group(n, n, n, &r.T2, 0, &r.T2, 1);  // T^4 = T^2 T^2
-    g4.epi.O = as_out(r.T4);
+    g4.epi.O = as_out(r.T4, false);
     GEMM_TRY(launch_gemm(&g4, 1, count, pr, st));
     GemmGroup gm = group(n, n, n, &r.T4, 0, &Mp[cm], 1);  // M' = T^4 M, next T = 1.25 I - 0.25 M'
-    gm.epi.O = as_out(Mp[1 - cm]);
-    gm.epi.X = as_out(r.T);
+    gm.epi.O = as_out(Mp[1 - cm], false);
+    gm.epi.X = as_out(r.T, false);
     gm.epi.alpha2 = -0.25f;
     gm.epi.gamma2 = 1.25f;
     GEMM_TRY(launch_gemm(&gm, 1, count, pr, st));
@@ -361,6 +371,7 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   Planes& S = r.Y[0];
   Planes* Bk1 = &r.Z[0];
   Planes* Bk2 = &r.Z[1];
+  Planes* Bk = &r.T;
   if (degree == 0) {
     GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[0], nullptr, *Bk2, pr, st));
     GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, X, status, st));
@@ -378,17 +389,19 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, (float)(4 * c[degree]), 0.f,
                             (float)(c[degree - 1] - 2 * c[degree]), scale, *Bk1, pr, st));
   for (int k = degree - 2; k >= 1; --k) {
-    // B_k = c_k I + 2 S B_{k+1} - B_{k+2}, written over B_{k+2}
+    // B_k = c_k I + 2 S B_{k+1} - B_{k+2}; three buffers, so that no launch
+    // writes a matrix it reads
     GemmGroup g = group(n, n, n, &S, 0, Bk1, 1);
     g.epi.alpha = 2.f;
     g.epi.beta = -1.f;
     g.epi.gamma = (float)c[k];
     g.epi.C = as_c(*Bk2);
-    g.epi.O = as_out(*Bk2);
+    g.epi.O = as_out(*Bk);
     GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
-    Planes* t = Bk1;
-    Bk1 = Bk2;
-    Bk2 = t;
+    Planes* t = Bk2;
+    Bk2 = Bk1;
+    Bk1 = Bk;
+    Bk = t;
   }
   // result = c_0 I + S B_1 - B_2, times s^(-1/4)
   GemmGroup g = group(n, n, n, &S, 0, Bk1, 1);
@@ -812,7 +825,7 @@ shp_status shampoo_precondition(const shp_plan* plan, const float* const* roots,
     CUDA_TRY(launch_to_planes(roots[rb], n, (long long)n * n, plan->dev + plan->off_ridx[g], cnt, n, n, 1.f, 0.f, 0.f,
                               nullptr, b.XR, pr, st));
     GemmGroup g1 = group(m, n, n, &b.G, 0, &b.XR, 1);  // P = G X_R
-    g1.epi.O = as_out(b.P);
+    g1.epi.O = as_out(b.P, false);
     cudaError_t e = launch_gemm(&g1, 1, cnt, pr, st);
     if (e != cudaSuccess) return fail(SHP_ERR_CUDA, "precondition GEMM 1: %s", cudaGetErrorString(e));
     GemmGroup g2 = group(m, n, m, &b.XL, 0, &b.P, 1);  // D = X_L P

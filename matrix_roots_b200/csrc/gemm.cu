@@ -12,15 +12,17 @@
 //   warps 0-7   two draining warpgroups (warp w reads TMEM lanes 32*(w%4)..,
 //               group h owns columns [h*BN/2, (h+1)*BN/2) of the tile)
 // The tensor core's FP32 accumulation error grows with the number of
-// products chained into one accumulator, so each K-block (one 128-byte row
-// of K: 32 tf32 or 64 f16/bf16 elements, 4 MMA slices) goes into its own
-// slot of a 4-deep TMEM ring; the draining warps add every slot into fp32
-// registers (round to nearest) and release it.  In FP32 mode (three TF32
-// passes on hi/lo operand splits) the small correction products lo*hi and
-// hi*lo are issued before hi*hi, so only the 4 hi*hi additions of a K-block
-// happen at the scale of the full partial sum.  The epilogue transposes
-// 32x32 blocks through shared memory so that reads of C and writes of the
-// output planes are 128-byte coalesced.
+// products chained into one accumulator, so partial products go into the
+// slots of a 4-deep TMEM ring that the draining warps add into fp32
+// registers (round to nearest) and release.  FP32 mode runs three fp16
+// passes on a scaled hi / lo split of each operand (x * 2^e = hi + lo *
+// 2^-11, e per matrix): per 32 K it issues the correction products lo*hi and
+// hi*lo into a fresh slot, then hi*hi with the input-D scale 2^-11 on the
+// first, so the corrections enter at their true weight.  Every output plane
+// set in that mode gets its exponent from a bound on its values and records
+// its max |value| for the next product.  The epilogue transposes 32x32
+// blocks through shared memory so that reads of C and writes of the output
+// planes are 128-byte (or 16-byte-per-lane) coalesced.
 #include <atomic>
 #include <cstdio>
 #include <mutex>
@@ -89,9 +91,9 @@ struct Cfg {
   static constexpr int B_TILE = BN * 128;
   static constexpr int STAGE_BYTES = NPL * (A_TILE + B_TILE);
   static constexpr int NBUF = 4;
-  // K-blocks accumulated in one TMEM slot before it is drained: every
-  // K-block in FP32 mode (accuracy), four in the one-pass modes, whose
-  // operand rounding (2^-11) dwarfs the accumulation error
+  // K-blocks accumulated in one TMEM slot before it is drained in the
+  // one-pass modes, whose operand rounding (2^-11) dwarfs the accumulation
+  // error; FP32 mode instead drains every half K-block (32 K), for accuracy
   static constexpr int DRAIN = (NPASS == 3) ? 1 : 4;
   static constexpr int TCOLS = NBUF * BN;
   static constexpr int THREADS = 320;
@@ -102,13 +104,6 @@ struct Cfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + RESERVED;
   static_assert(STAGES >= 2 && TCOLS <= 512 && BN <= 128, "tile does not fit");
 };
-
-__device__ __forceinline__ void store_h16(void* base, long long off, float v, int bf) {
-  if (bf)
-    reinterpret_cast<__nv_bfloat16*>(base)[off] = __float2bfloat16_rn(v);
-  else
-    reinterpret_cast<__half*>(base)[off] = __float2half_rn(v);
-}
 
 struct Tile {
   int grp, b, m0, n0, nk;
@@ -131,43 +126,93 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN, 
 // One output plane set with its pointers already offset to (row0, col).
 struct OutPtrs {
   float* f32;
-  float* lo;
   void* h16;
+  __half* h16lo;  // non-null: h16 / h16lo hold the scaled fp16 hi / lo split
   int bf;
   int ld;
+  float sc;  // 2^exp of the split
 };
 
-__device__ __forceinline__ OutPtrs out_ptrs(const EpiOut& o, int ob, int row0, int col) {
+__device__ __forceinline__ OutPtrs out_ptrs(const EpiOut& o, int ob, int row0, int col, float sc) {
   OutPtrs r;
   const long long off = (long long)ob * o.bs + (long long)row0 * o.ld + col;
   r.f32 = o.f32 ? o.f32 + off : nullptr;
-  r.lo = o.lo ? o.lo + off : nullptr;
   r.h16 = o.h16 ? (o.h16_bf ? (void*)(reinterpret_cast<__nv_bfloat16*>(o.h16) + off)
                             : (void*)(reinterpret_cast<__half*>(o.h16) + off))
                 : nullptr;
+  r.h16lo = o.h16lo ? reinterpret_cast<__half*>(o.h16lo) + off : nullptr;
   r.bf = o.h16_bf;
   r.ld = o.ld;
+  r.sc = sc;
   return r;
+}
+
+// Per-tile epilogue constants of one problem and matrix.
+struct EpiCtx {
+  int ob;
+  float mult, alpha, beta, gamma, alpha2, beta2, gamma2;
+  bool has_x, need_c;
+  float scO, scX;
+};
+
+// r0 = alpha*AB + beta*C + gamma*I with the operand scales undone; the
+// scale exponent of a split output comes from the bound
+//   |r0| <= |alpha| K max|A| max|B| + |beta| max|C| + |gamma|
+// (and the same for the aux output), and is stored for the next GEMM.
+__device__ __forceinline__ EpiCtx make_ctx(const GroupDev& g, int b, bool write_exp) {
+  EpiCtx c;
+  c.ob = g.o_idx ? g.o_idx[b] : b;
+  c.mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+  c.has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
+  c.need_c = (g.beta != 0.f) || (c.has_x && g.beta2 != 0.f);
+  c.alpha = g.alpha;
+  c.beta = g.beta;
+  c.gamma = g.gamma;
+  c.alpha2 = g.alpha2;
+  c.beta2 = g.beta2;
+  c.gamma2 = g.gamma2;
+  c.scO = 1.f;
+  c.scX = 1.f;
+  if (g.a_exp) {
+    const int ai = g.a_idx ? g.a_idx[b] : b;
+    const int bi = g.b_idx ? g.b_idx[b] : b;
+    c.alpha = g.alpha * pow2f(-g.a_exp[ai]) * pow2f(-g.b_exp[bi]);
+    const float cmax = (c.need_c && g.C.amax) ? g.C.amax[c.ob] : 0.f;
+    const float r0 = fabsf(g.alpha) * (float)g.K * g.a_amax[ai] * g.b_amax[bi] + fabsf(g.beta) * cmax + fabsf(g.gamma);
+    if (g.O.h16lo) {
+      const int e = split_exp(fabsf(c.mult) * r0);
+      c.scO = pow2f(e);
+      if (write_exp) g.O.exp[c.ob] = e;
+    }
+    if (c.has_x && g.X.h16lo) {
+      const int e = split_exp(fabsf(c.mult) * (fabsf(g.alpha2) * r0 + fabsf(g.beta2) * cmax + fabsf(g.gamma2)));
+      c.scX = pow2f(e);
+      if (write_exp) g.X.exp[c.ob] = e;
+    }
+  }
+  return c;
 }
 
 // Stores rows [r0, r0 + 8) of values v (rows >= rmax skipped) into one
 // output plane set; the format tests are uniform and sit outside the rows.
 __device__ __forceinline__ void put_rows(const OutPtrs& o, int r0, int rmax, const float (&v)[8]) {
   const long long ld = o.ld;
-  if (o.lo) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (r0 + i < rmax) {
-        const float hi = tf32_round(v[i]);
-        o.f32[(r0 + i) * ld] = hi;
-        o.lo[(r0 + i) * ld] = v[i] - hi;
-      }
-  } else if (o.f32) {
+  if (o.f32) {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       if (r0 + i < rmax) o.f32[(r0 + i) * ld] = v[i];
   }
-  if (o.h16) {
+  if (o.h16lo) {
+    __half* h = reinterpret_cast<__half*>(o.h16);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (r0 + i < rmax) {
+        __half hi, lo;
+        split16(v[i] * o.sc, hi, lo);
+        h[(r0 + i) * ld] = hi;
+        o.h16lo[(r0 + i) * ld] = lo;
+      }
+  } else if (o.h16) {
     if (o.bf) {
       __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(o.h16);
 #pragma unroll
@@ -186,26 +231,14 @@ __device__ __forceinline__ void put_rows(const OutPtrs& o, int r0, int rmax, con
 // in `stage` (element (r, c) at r*32 + (c ^ r)): lane = column, so every
 // load of C and every store of an output plane is one 128-byte segment.
 // Rows go in groups of 8: values first, then the stores of the group.
-__device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row0, int col, const float* stage,
-                                               int lane, float& ss, int& bad) {
+__device__ __forceinline__ void epilogue_block(const GroupDev& g, const EpiCtx& x, int row0, int col,
+                                               const float* stage, int lane, float& ss, int& bad, float& mo,
+                                               float& mx) {
   if (col >= g.N) return;
-  const int ob = g.o_idx ? g.o_idx[b] : b;
-  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
-  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
-  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
-  const OutPtrs O = out_ptrs(g.O, ob, row0, col);
-  const OutPtrs X = has_x ? out_ptrs(g.X, ob, row0, col) : O;
-  const float* cf = nullptr;
-  const float* cl = nullptr;
-  long long cld = 0;
-  if (need_c) {
-    const long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
-    cf = g.C.f32 + coff;
-    cl = g.C.lo ? g.C.lo + coff : nullptr;
-    cld = g.C.ld;
-  }
-  const float alpha = g.alpha, beta = g.beta, gamma = g.gamma;
-  const float alpha2 = g.alpha2, beta2 = g.beta2, gamma2 = g.gamma2;
+  const OutPtrs O = out_ptrs(g.O, x.ob, row0, col, x.scO);
+  const OutPtrs X = x.has_x ? out_ptrs(g.X, x.ob, row0, col, x.scX) : O;
+  const float* cf = x.need_c ? g.C.f32 + (long long)x.ob * g.C.bs + (long long)row0 * g.C.ld + col : nullptr;
+  const long long cld = g.C.ld;
   const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
   const int dr = col - row0;  // the diagonal sits in row dr of this block
 #pragma unroll 1
@@ -213,26 +246,28 @@ __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row
     float cv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) cv[i] = 0.f;
-    if (need_c) {
+    if (x.need_c) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        if (r0 + i < rmax) cv[i] = cf[(r0 + i) * cld] + (cl ? cl[(r0 + i) * cld] : 0.f);
+        if (r0 + i < rmax) cv[i] = cf[(r0 + i) * cld];
     }
     float v[8], xv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = r0 + i;
       const float diag = (r == dr) ? 1.f : 0.f;
-      const float q0 = alpha * stage[r * 32 + (lane ^ r)] + beta * cv[i] + gamma * diag;
-      v[i] = q0 * mult;
-      xv[i] = mult * (alpha2 * q0 + beta2 * cv[i] + gamma2 * diag);
+      const float q0 = x.alpha * stage[r * 32 + (lane ^ r)] + x.beta * cv[i] + x.gamma * diag;
+      v[i] = q0 * x.mult;
+      xv[i] = x.mult * (x.alpha2 * q0 + x.beta2 * cv[i] + x.gamma2 * diag);
       if (r < rmax) {
         ss += v[i] * v[i];
         bad |= !isfinite(v[i]);
+        mo = fmaxf(mo, fabsf(v[i]));
+        mx = fmaxf(mx, fabsf(xv[i]));
       }
     }
     put_rows(O, r0, rmax, v);
-    if (has_x) put_rows(X, r0, rmax, xv);
+    if (x.has_x) put_rows(X, r0, rmax, xv);
   }
 }
 
@@ -240,19 +275,25 @@ __device__ __forceinline__ void epilogue_block(const GroupDev& g, int b, int row
 // `stage` as rows of eight float4 slots, slot j of row r at r*8 + (j ^ (r&7));
 // each lane handles four consecutive columns of one row, a warp four rows
 // per step, so each store is a 128-byte row segment per eight lanes.
+__device__ __forceinline__ uint2 pack_half4(__half a, __half b, __half c, __half d) {
+  __half2 p = __halves2half2(a, b), q = __halves2half2(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&p);
+  u.y = *reinterpret_cast<uint32_t*>(&q);
+  return u;
+}
+
 __device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) {
-  if (o.lo) {
-    float4 hi;
-    hi.x = tf32_round(v.x);
-    hi.y = tf32_round(v.y);
-    hi.z = tf32_round(v.z);
-    hi.w = tf32_round(v.w);
-    *reinterpret_cast<float4*>(o.f32 + off) = hi;
-    *reinterpret_cast<float4*>(o.lo + off) = make_float4(v.x - hi.x, v.y - hi.y, v.z - hi.z, v.w - hi.w);
-  } else if (o.f32) {
-    *reinterpret_cast<float4*>(o.f32 + off) = v;
-  }
-  if (o.h16) {
+  if (o.f32) *reinterpret_cast<float4*>(o.f32 + off) = v;
+  if (o.h16lo) {
+    __half h0, h1, h2, h3, l0, l1, l2, l3;
+    split16(v.x * o.sc, h0, l0);
+    split16(v.y * o.sc, h1, l1);
+    split16(v.z * o.sc, h2, l2);
+    split16(v.w * o.sc, h3, l3);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) = pack_half4(h0, h1, h2, h3);
+    *reinterpret_cast<uint2*>(o.h16lo + off) = pack_half4(l0, l1, l2, l3);
+  } else if (o.h16) {
     if (o.bf) {
       __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
       uint2 u;
@@ -260,37 +301,24 @@ __device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) 
       u.y = *reinterpret_cast<uint32_t*>(&b);
       *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(o.h16) + off) = u;
     } else {
-      __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
-      uint2 u;
-      u.x = *reinterpret_cast<uint32_t*>(&a);
-      u.y = *reinterpret_cast<uint32_t*>(&b);
-      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) = u;
+      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) =
+          pack_half4(__float2half_rn(v.x), __float2half_rn(v.y), __float2half_rn(v.z), __float2half_rn(v.w));
     }
   }
 }
 
-__device__ __forceinline__ void epilogue_block4(const GroupDev& g, int b, int row0, int col0, const float4* stage,
-                                                int lane, float& ss, int& bad) {
+__device__ __forceinline__ float max4(float4 v) { return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))); }
+
+__device__ __forceinline__ void epilogue_block4(const GroupDev& g, const EpiCtx& x, int row0, int col0,
+                                                const float4* stage, int lane, float& ss, int& bad, float& mo,
+                                                float& mx) {
   const int cq = lane & 7;
   const int col = col0 + 4 * cq;
   if (col >= g.N) return;
-  const int ob = g.o_idx ? g.o_idx[b] : b;
-  const float mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
-  const bool has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
-  const bool need_c = (g.beta != 0.f) || (has_x && g.beta2 != 0.f);
-  const OutPtrs O = out_ptrs(g.O, ob, row0, col);
-  const OutPtrs X = has_x ? out_ptrs(g.X, ob, row0, col) : O;
-  const float* cf = nullptr;
-  const float* cl = nullptr;
-  long long cld = 0;
-  if (need_c) {
-    const long long coff = (long long)ob * g.C.bs + (long long)row0 * g.C.ld + col;
-    cf = g.C.f32 + coff;
-    cl = g.C.lo ? g.C.lo + coff : nullptr;
-    cld = g.C.ld;
-  }
-  const float alpha = g.alpha, beta = g.beta, gamma = g.gamma;
-  const float alpha2 = g.alpha2, beta2 = g.beta2, gamma2 = g.gamma2;
+  const OutPtrs O = out_ptrs(g.O, x.ob, row0, col, x.scO);
+  const OutPtrs X = x.has_x ? out_ptrs(g.X, x.ob, row0, col, x.scX) : O;
+  const float* cf = x.need_c ? g.C.f32 + (long long)x.ob * g.C.bs + (long long)row0 * g.C.ld + col : nullptr;
+  const long long cld = g.C.ld;
   const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
 #pragma unroll 2
   for (int it = 0; it < 8; ++it) {
@@ -298,34 +326,26 @@ __device__ __forceinline__ void epilogue_block4(const GroupDev& g, int b, int ro
     if (r >= rmax) continue;
     const float4 a = stage[r * 8 + (cq ^ (r & 7))];
     float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (need_c) {
-      c = *reinterpret_cast<const float4*>(cf + r * cld);
-      if (cl) {
-        const float4 l = *reinterpret_cast<const float4*>(cl + r * cld);
-        c.x += l.x;
-        c.y += l.y;
-        c.z += l.z;
-        c.w += l.w;
-      }
-    }
+    if (x.need_c) c = *reinterpret_cast<const float4*>(cf + r * cld);
     const int e = row0 + r - col;  // component on the diagonal, if 0..3
     const float d0 = e == 0 ? 1.f : 0.f, d1 = e == 1 ? 1.f : 0.f, d2 = e == 2 ? 1.f : 0.f, d3 = e == 3 ? 1.f : 0.f;
     float4 q;
-    q.x = alpha * a.x + beta * c.x + gamma * d0;
-    q.y = alpha * a.y + beta * c.y + gamma * d1;
-    q.z = alpha * a.z + beta * c.z + gamma * d2;
-    q.w = alpha * a.w + beta * c.w + gamma * d3;
-    const float4 v = make_float4(q.x * mult, q.y * mult, q.z * mult, q.w * mult);
-    const long long off = (long long)r * O.ld;
-    put4(O, off, v);
+    q.x = x.alpha * a.x + x.beta * c.x + x.gamma * d0;
+    q.y = x.alpha * a.y + x.beta * c.y + x.gamma * d1;
+    q.z = x.alpha * a.z + x.beta * c.z + x.gamma * d2;
+    q.w = x.alpha * a.w + x.beta * c.w + x.gamma * d3;
+    const float4 v = make_float4(q.x * x.mult, q.y * x.mult, q.z * x.mult, q.w * x.mult);
+    put4(O, (long long)r * O.ld, v);
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
-    if (has_x) {
-      const float4 xv = make_float4(mult * (alpha2 * q.x + beta2 * c.x + gamma2 * d0),
-                                    mult * (alpha2 * q.y + beta2 * c.y + gamma2 * d1),
-                                    mult * (alpha2 * q.z + beta2 * c.z + gamma2 * d2),
-                                    mult * (alpha2 * q.w + beta2 * c.w + gamma2 * d3));
+    mo = fmaxf(mo, max4(v));
+    if (x.has_x) {
+      const float4 xv = make_float4(x.mult * (x.alpha2 * q.x + x.beta2 * c.x + x.gamma2 * d0),
+                                    x.mult * (x.alpha2 * q.y + x.beta2 * c.y + x.gamma2 * d1),
+                                    x.mult * (x.alpha2 * q.z + x.beta2 * c.z + x.gamma2 * d2),
+                                    x.mult * (x.alpha2 * q.w + x.beta2 * c.w + x.gamma2 * d3));
       put4(X, (long long)r * X.ld, xv);
+      mx = fmaxf(mx, max4(xv));
     }
   }
 }
@@ -477,35 +497,55 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         const uint64_t a_step = (g.a_mn ? KSTEP_MN : KSTEP_K) >> 4;
         const uint64_t b_step = (g.b_mn ? KSTEP_MN : KSTEP_K) >> 4;
         bool ok = true;
-        for (int kb = 0; kb < x.nk; ++kb) {
-          if (!mbar_wait(full0 + 8 * st.i, st.ph) || (in_slot == 0 && !mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1))) {
+        for (int kb = 0; kb < x.nk && ok; ++kb) {
+          if (!mbar_wait(full0 + 8 * st.i, st.ph)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint64_t so = (uint64_t)(st.i * (C::STAGE_BYTES >> 4));
           const uint64_t ad = a0 + so, bd = b0 + so;
-          const uint32_t d = tmem + sl.i * BN;
           if constexpr (NPASS == 3) {
-            // the 8 small correction products first, while the slot is small
+            // two TMEM slots per K-block, 32 K each: in each, the correction
+            // products lo*hi and hi*lo first (in units of 2^-11), then hi*hi,
+            // the first of which scales the slot by 2^-11
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-              mma<KIND>(d, ad + (C::A_TILE >> 4) + ks * a_step, bd + ks * b_step, idesc, ks ? 1u : 0u);
-              mma<KIND>(d, ad + ks * a_step, bd + (C::B_TILE >> 4) + ks * b_step, idesc, 1u);
+            for (int hs = 0; hs < KS / 2; ++hs) {
+              if (!mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem + sl.i * BN;
+#pragma unroll
+              for (int ks = 2 * hs; ks < 2 * hs + 2; ++ks) {
+                mma<KIND>(d, ad + (C::A_TILE >> 4) + ks * a_step, bd + ks * b_step, idesc, ks > 2 * hs ? 1u : 0u);
+                mma<KIND>(d, ad + ks * a_step, bd + (C::B_TILE >> 4) + ks * b_step, idesc, 1u);
+              }
+              mma_f16_scale11(d, ad + 2 * hs * a_step, bd + 2 * hs * b_step, idesc);
+              mma<KIND>(d, ad + (2 * hs + 1) * a_step, bd + (2 * hs + 1) * b_step, idesc, 1u);
+              tc_commit(tfull0 + 8 * sl.i);
+              sl.template next<NB>();
             }
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, 1u);
+            if (!ok) break;
+            tc_commit(empty0 + 8 * st.i);
+            st.template next<S>();
           } else {
+            if (in_slot == 0 && !mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + sl.i * BN;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks)
               mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, (in_slot | ks) ? 1u : 0u);
-          }
-          tc_commit(empty0 + 8 * st.i);
-          st.template next<S>();
-          if (++in_slot == DR || kb == x.nk - 1) {
-            tc_commit(tfull0 + 8 * sl.i);
-            sl.template next<NB>();
-            in_slot = 0;
+            tc_commit(empty0 + 8 * st.i);
+            st.template next<S>();
+            if (++in_slot == DR || kb == x.nk - 1) {
+              tc_commit(tfull0 + 8 * sl.i);
+              sl.template next<NB>();
+              in_slot = 0;
+            }
           }
         }
         if (!ok) {
@@ -531,7 +571,7 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
 #pragma unroll
       for (int i = 0; i < HC; ++i) acc[i] = 0.f;
       bool ok = true;
-      const int nslots = (x.nk + DR - 1) / DR;
+      const int nslots = NPASS == 3 ? x.nk * (KS / 2) : (x.nk + DR - 1) / DR;
       for (int u = 0; u < nslots; ++u) {
         ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * sl.i, sl.ph));
         if (!ok) {
@@ -553,8 +593,9 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       }
       if (!ok) break;
       const GroupDev& g = p.g[x.grp];
+      const EpiCtx ec = make_ctx(g, x.b, lane == 0);
       int bad = 0;
-      float ss = 0.f;
+      float ss = 0.f, mo = 0.f, mx = 0.f;
       if (g.vec4) {
         float4* stage4 = reinterpret_cast<float4*>(stage);
 #pragma unroll
@@ -564,7 +605,7 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
             stage4[lane * 8 + (j ^ (lane & 7))] = make_float4(acc[ch * 32 + 4 * j], acc[ch * 32 + 4 * j + 1],
                                                               acc[ch * 32 + 4 * j + 2], acc[ch * 32 + 4 * j + 3]);
           __syncwarp();
-          epilogue_block4(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32, stage4, lane, ss, bad);
+          epilogue_block4(g, ec, x.m0 + q * 32, x.n0 + h * HC + ch * 32, stage4, lane, ss, bad, mo, mx);
           __syncwarp();
         }
       } else {
@@ -573,16 +614,28 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
 #pragma unroll
           for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = acc[ch * 32 + c];
           __syncwarp();
-          epilogue_block(g, x.b, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad);
+          epilogue_block(g, ec, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad, mo, mx);
           __syncwarp();
         }
       }
       if (g.sumsq) {
 #pragma unroll
         for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) atomicAdd(g.sumsq + (g.o_idx ? g.o_idx[x.b] : x.b), ss);
+        if (lane == 0) atomicAdd(g.sumsq + ec.ob, ss);
       }
-      if (g.status && bad) atomicOr(g.status + (g.o_idx ? g.o_idx[x.b] : x.b), 1);
+      // max |value| of the split outputs, for the scale bound of the next GEMM
+      // (non-negative floats order like their bit patterns)
+      if (g.O.amax) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mo = fmaxf(mo, __shfl_xor_sync(0xffffffffu, mo, o));
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(g.O.amax) + ec.ob, __float_as_uint(mo));
+      }
+      if (ec.has_x && g.X.amax) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(g.X.amax) + ec.ob, __float_as_uint(mx));
+      }
+      if (g.status && bad) atomicOr(g.status + ec.ob, 1);
     }
   }
 
@@ -680,7 +733,7 @@ cudaError_t run(GemmParams& prm, cudaStream_t stream) {
 
 cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec prec, cudaStream_t stream) {
   if (ngroups < 1 || ngroups > 2 || batch < 1) return cudaErrorInvalidValue;
-  const int kind = (prec == P_FP16) ? 1 : (prec == P_BF16) ? 2 : 0;
+  const int kind = (prec == P_FP16 || prec == P_FP32) ? 1 : (prec == P_BF16) ? 2 : 0;
   const int npass = (prec == P_FP32) ? 3 : 1;
   const int esz = kind ? 2 : 4;
   const int bke = 128 / esz;
@@ -707,24 +760,37 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
     d.b_mn = G.b_mn;
     d.a_idx = G.a_idx;
     d.b_idx = G.b_idx;
+    if (npass == 3) {
+      if (!G.A->exp || !G.B->exp || !G.A->amax || !G.B->amax || !G.A->h16lo || !G.B->h16lo)
+        return cudaErrorInvalidValue;
+      d.a_exp = G.A->exp;
+      d.b_exp = G.B->exp;
+      d.a_amax = G.A->amax;
+      d.b_amax = G.B->amax;
+    } else {
+      d.a_exp = d.b_exp = nullptr;
+      d.a_amax = d.b_amax = nullptr;
+      // the split output format needs the operand scales
+      if (d.O.h16lo || d.X.h16lo) return cudaErrorInvalidValue;
+    }
     prm.g[i] = d;
     prm.a4d[i] = G.a_mn && G.A->ld % bke == 0;
     {
       auto al16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; };
       auto al8 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 7u) == 0; };
       auto ok_out = [&](const EpiOut& o) {
-        return (o.ld % 4 == 0) && (o.bs % 4 == 0) && al16(o.f32) && al16(o.lo) && al8(o.h16);
+        return (o.ld % 4 == 0) && (o.bs % 4 == 0) && al16(o.f32) && al8(o.h16) && al8(o.h16lo);
       };
       const bool has_x = d.X.f32 || d.X.h16;
       const bool need_c = d.beta != 0.f || (has_x && d.beta2 != 0.f);
       bool v = G.N % 4 == 0 && ok_out(d.O) && (!has_x || ok_out(d.X));
-      if (need_c) v = v && d.C.ld % 4 == 0 && d.C.bs % 4 == 0 && al16(d.C.f32) && al16(d.C.lo);
+      if (need_c) v = v && d.C.ld % 4 == 0 && d.C.bs % 4 == 0 && al16(d.C.f32);
       prm.g[i].vec4 = v ? 1 : 0;
     }
     prm.b4d[i] = G.b_mn && G.B->ld % bke == 0;
     for (int pl = 0; pl < (npass == 3 ? 2 : 1); ++pl) {
-      const void* abase = kind ? G.A->h16 : (pl ? (const void*)G.A->lo : (const void*)G.A->f32);
-      const void* bbase = kind ? G.B->h16 : (pl ? (const void*)G.B->lo : (const void*)G.B->f32);
+      const void* abase = kind ? (pl ? G.A->h16lo : G.A->h16) : (const void*)G.A->f32;
+      const void* bbase = kind ? (pl ? G.B->h16lo : G.B->h16) : (const void*)G.B->f32;
       if (prm.a4d[i]) {
         if (!make_map_4d(&prm.tmA[i][pl], abase, dt, esz, *G.A, bke, 128 / bke, kind == 0))
           return cudaErrorInvalidValue;
@@ -746,7 +812,16 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
   }
   if (total > (1ll << 30)) return cudaErrorInvalidValue;
   prm.total_tiles = (int)total;
-  if (kind == 0 && npass == 3) return BN == 64 ? run<0, 3, 64>(prm, stream) : run<0, 3, 128>(prm, stream);
+  // the outputs' max |value| accumulate by atomic max from zero
+  for (int i = 0; i < ngroups; ++i) {
+    const EpiOut* outs[2] = {&groups[i].epi.O, &groups[i].epi.X};
+    for (const EpiOut* o : outs)
+      if (o->amax && o->amax_n > 0) {
+        cudaError_t e = cudaMemsetAsync(o->amax, 0, sizeof(float) * o->amax_n, stream);
+        if (e != cudaSuccess) return e;
+      }
+  }
+  if (npass == 3) return BN == 64 ? run<1, 3, 64>(prm, stream) : run<1, 3, 128>(prm, stream);
   if (kind == 0) return BN == 64 ? run<0, 1, 64>(prm, stream) : run<0, 1, 128>(prm, stream);
   if (kind == 1) return BN == 64 ? run<1, 1, 64>(prm, stream) : run<1, 1, 128>(prm, stream);
   return BN == 64 ? run<2, 1, 64>(prm, stream) : run<2, 1, 128>(prm, stream);

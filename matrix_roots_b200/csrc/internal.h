@@ -11,30 +11,38 @@ enum Prec : int { P_FP32 = 0, P_TF32 = 1, P_FP16 = 2, P_BF16 = 3 };
 
 // A stack of `count` matrices (rows x cols, leading dimension ld, batch
 // stride bs elements) stored in the planes a tensor-core pass reads:
-//   FP32 : f32 = tf32-rounded high part, lo = remainder (value = f32 + lo)
+//   FP32 : per matrix b a power-of-two scale 2^exp[b]; with y = x * 2^e,
+//          h16 = fp16(y) and h16lo = fp16((y - h16) * 2^11), so that
+//          y = h16 + h16lo * 2^-11 to about 22 bits; f32 = x (may be null);
+//          amax[b] = max |x| of the matrix
 //   TF32 : f32 = full value
 //   FP16 / BF16 : f32 = full value (may be null), h16 = half copy
 struct Planes {
   float* f32 = nullptr;
-  float* lo = nullptr;
   void* h16 = nullptr;
+  void* h16lo = nullptr;
+  int* exp = nullptr;
+  float* amax = nullptr;
   int h16_bf = 0;  // 1 when h16 holds bfloat16
   int rows = 0, cols = 0, ld = 0;
   long long bs = 0;
   int count = 0;
 };
 
-// Epilogue input C (value = f32 + lo) and outputs.
+// Epilogue input C (its full fp32 value) and outputs.
 struct EpiC {
   const float* f32 = nullptr;
-  const float* lo = nullptr;
+  const float* amax = nullptr;  // per-matrix max |C| (FP32 planes), for the output scale bound
   int ld = 0;
   long long bs = 0;
 };
 struct EpiOut {
-  float* f32 = nullptr;  // full value, or the tf32-rounded high part when lo != null
-  float* lo = nullptr;
-  void* h16 = nullptr;
+  float* f32 = nullptr;  // full value (may be null)
+  void* h16 = nullptr;   // half copy, or the scaled fp16 high part when h16lo != null
+  void* h16lo = nullptr;
+  int* exp = nullptr;
+  float* amax = nullptr;
+  int amax_n = 0;  // entries of amax, cleared before the launch
   int h16_bf = 0;
   int ld = 0;
   long long bs = 0;
@@ -52,6 +60,11 @@ struct GroupDev {
   int a_mn = 0, b_mn = 0;  // 1: operand stored MN-major (K rows x M/N cols)
   const int* a_idx = nullptr;
   const int* b_idx = nullptr;
+  // FP32 planes of the operands: scale exponents and max |x|
+  const int* a_exp = nullptr;
+  const int* b_exp = nullptr;
+  const float* a_amax = nullptr;
+  const float* b_amax = nullptr;
   const int* o_idx = nullptr;
   float alpha = 1.f, beta = 0.f, gamma = 0.f;
   const float* bscale = nullptr;
@@ -91,14 +104,16 @@ struct GemmGroup {
   GroupDev epi;  // epilogue part (M/N/K/majors/idx filled by the launcher)
 };
 
-// prec: the arithmetic of the tensor-core passes (FP32 = 3 x TF32 split).
+// prec: the arithmetic of the tensor-core passes (FP32 = three fp16 passes on
+// the scaled hi / lo split).
 cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec prec, cudaStream_t stream);
 
 // ---- elementwise / reduction kernels (kernels.cu) ------------------------
 
 // dst = (alpha/s_b) * src + (eps/s_b + delta) * I, written in the planes of
 // `dst` for precision `prec`.  src: count matrices rows x cols (ld, bs),
-// optional batch index map; s_b = scale[b] or 1.
+// optional batch index map; s_b = scale[b] or 1.  For FP32 planes a first
+// pass finds max |dst| per matrix, which fixes the scale exponent.
 cudaError_t launch_to_planes(const float* src, int src_ld, long long src_bs, const int* src_idx, int count,
                              int rows, int cols, float alpha, float eps, float delta, const float* scale,
                              const Planes& dst, Prec prec, cudaStream_t stream);

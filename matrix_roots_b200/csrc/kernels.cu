@@ -14,19 +14,52 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ void put(const Planes& d, long long off, float v, int prec) {
-  if (prec == P_FP32) {
-    const float hi = tf32_round(v);
-    d.f32[off] = hi;
-    d.lo[off] = v - hi;
-    return;
-  }
+__device__ __forceinline__ void put(const Planes& d, long long off, float v, int prec, float sc) {
   if (d.f32) d.f32[off] = v;
-  if (prec == P_FP16 || prec == P_BF16) {
+  if (prec == P_FP32) {
+    __half hi, lo;
+    split16(v * sc, hi, lo);
+    reinterpret_cast<__half*>(d.h16)[off] = hi;
+    reinterpret_cast<__half*>(d.h16lo)[off] = lo;
+  } else if (prec == P_FP16 || prec == P_BF16) {
     if (d.h16_bf)
       reinterpret_cast<__nv_bfloat16*>(d.h16)[off] = __float2bfloat16_rn(v);
     else
       reinterpret_cast<__half*>(d.h16)[off] = __float2half_rn(v);
+  }
+}
+
+// amax[b] = max |(alpha/s_b) src_b + (eps/s_b + delta) I| (amax cleared before).
+__global__ void amax_affine_kernel(const float* __restrict__ src, int src_ld, long long src_bs,
+                                   const int* __restrict__ src_idx, int rows, int cols, float alpha, float eps,
+                                   float delta, const float* __restrict__ scale, float* __restrict__ amax) {
+  __shared__ float red[32];
+  const int b = blockIdx.y;
+  const long long sb = src_idx ? src_idx[b] : b;
+  const float inv_s = scale ? 1.f / scale[b] : 1.f;
+  const float a = alpha * inv_s;
+  const float d = eps * inv_s + delta;
+  const float* s = src + sb * src_bs;
+  const long long total = (long long)rows * cols;
+  float m = 0.f;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(e / cols);
+    const int c = (int)(e - (long long)r * cols);
+    const float x = (a != 0.f) ? a * s[(long long)r * src_ld + c] : 0.f;
+    m = fmaxf(m, fabsf(x + (r == c ? d : 0.f)));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = m;
+  __syncthreads();
+  if (w == 0) {
+    m = l < (int)(blockDim.x >> 5) ? red[l] : 0.f;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // non-negative floats order like their bit patterns
+    if (l == 0) atomicMax(reinterpret_cast<unsigned int*>(amax) + b, __float_as_uint(m));
   }
 }
 
@@ -40,6 +73,12 @@ __global__ void to_planes_kernel(const float* __restrict__ src, int src_ld, long
   const float d = eps * inv_s + delta;
   const float* s = src + sb * src_bs;
   const long long dbase = (long long)b * dst.bs;
+  float sc = 1.f;
+  if (prec == P_FP32) {
+    const int ex = split_exp(dst.amax[b]);
+    sc = pow2f(ex);
+    if (blockIdx.x == 0 && threadIdx.x == 0) dst.exp[b] = ex;
+  }
   const int per_row = cols;
   const long long total = (long long)rows * per_row;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
@@ -48,7 +87,7 @@ __global__ void to_planes_kernel(const float* __restrict__ src, int src_ld, long
     const int c = (int)(e - (long long)r * per_row);
     const float x = (a != 0.f) ? a * s[(long long)r * src_ld + c] : 0.f;  // a == 0: identity only
     const float v = x + (r == c ? d : 0.f);
-    put(dst, dbase + (long long)r * dst.ld + c, v, prec);
+    put(dst, dbase + (long long)r * dst.ld + c, v, prec, sc);
   }
 }
 
@@ -167,6 +206,13 @@ cudaError_t launch_to_planes(const float* src, int src_ld, long long src_bs, con
   const long long per = (long long)rows * cols;
   int gx = grid_for(per, kThreads * 8);
   dim3 grid(gx, count);
+  if (prec == P_FP32) {
+    cudaError_t e = cudaMemsetAsync(dst.amax, 0, sizeof(float) * count, stream);
+    if (e != cudaSuccess) return e;
+    amax_affine_kernel<<<grid, kThreads, 0, stream>>>(src, src_ld, src_bs, src_idx, rows, cols, alpha, eps, delta,
+                                                      scale, dst.amax);
+    count_launch();
+  }
   to_planes_kernel<<<grid, kThreads, 0, stream>>>(src, src_ld, src_bs, src_idx, rows, cols, alpha, eps, delta,
                                                   scale, dst, (int)prec);
   count_launch();

@@ -5,6 +5,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace shp {
@@ -123,6 +124,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint
       : "memory");
 }
 
+// D = A*B + D * 2^-11 (kind::f16, the input-D scale operand): adds the
+// high-part product to correction products accumulated in units of 2^-11.
+__device__ __forceinline__ void mma_f16_scale11(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.eq.u32 p, 1, 1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p, 11;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc)
+      : "memory");
+}
+
 // 32 lanes x 16 consecutive 32-bit columns: thread t of the warp receives
 // row (lane base + t), columns [col, col+16).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
@@ -175,10 +187,25 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t a_fmt, uint32_t b_f
          ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ float tf32_round(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
+// ---- scaled fp16 hi / lo split (FP32 mode operands) ----------------------
+
+// Exponent e such that |x| <= bound implies |x * 2^e| < 2^14 (fp16 holds it
+// with room to spare); 0 for a zero or non-finite bound.
+__device__ __forceinline__ int split_exp(float bound) {
+  if (!(bound > 0.f) || !(bound < 3.0e38f)) return 0;
+  int k;
+  frexpf(bound, &k);  // bound < 2^k
+  const int e = 14 - k;
+  return e < -100 ? -100 : (e > 100 ? 100 : e);
+}
+
+// 2^e as a float, exact for |e| <= 126.
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+// y = hi + lo * 2^-11 with hi = fp16(y), lo = fp16 of the scaled remainder.
+__device__ __forceinline__ void split16(float y, __half& hi, __half& lo) {
+  hi = __float2half_rn(y);
+  lo = __float2half_rn((y - __half2float(hi)) * 2048.f);
 }
 
 }  // namespace shp

@@ -154,9 +154,7 @@ __global__ void scaled_copy_kernel(Planes P, int n, const float* __restrict__ sc
        e += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(e / n), c = (int)(e - (long long)r * n);
     const long long off = (long long)b * P.bs + (long long)r * P.ld + c;
-    float x = P.f32[off];
-    if (P.lo) x += P.lo[off];
-    x *= mult;
+    const float x = P.f32[off] * mult;
     out[(long long)b * n * n + e] = x;
     bad |= !isfinite(x);
   }

@@ -157,6 +157,7 @@ void split_dim(int d, int B, std::vector<int>& out) {
 struct RootBufs {
   Planes Y[2], Z[2], T, T2, T4;
   double* sums = nullptr;
+  float* lmax = nullptr;  // max |L| per matrix, bounds the FP32 plane exponents
   float* fscale = nullptr;
   Planes A16, Vt, W;
 };
@@ -164,6 +165,7 @@ struct RootBufs {
 RootBufs carve_roots(Carver& c, int count, int n, int method, Prec pr, int scaling, int pi_vectors) {
   RootBufs r;
   r.sums = static_cast<double*>(c.take(sizeof(double) * count));
+  r.lmax = static_cast<float*>(c.take(sizeof(float) * count));
   if (method == SHP_METHOD_NDB) {
     for (int i = 0; i < 2; ++i) {
       r.Y[i] = make_planes(c, count, n, n, pr);
@@ -225,7 +227,7 @@ shp_status check_gemm(cudaError_t e, const char* what) {
 // Scale s_b of L_b (+ eps I): Frobenius norm or multi-power-iteration.
 shp_status compute_scale(const float* A, int count, int n, float eps_s, int scaling, int pi_vectors, int pi_iters,
                          const float* pi_starts, RootBufs& r, float* scale_out, cudaStream_t st) {
-  GEMM_TRY(launch_frob_sumsq(A, n, n, (long long)n * n, count, eps_s, r.sums, st));
+  GEMM_TRY(launch_frob_sumsq(A, n, n, (long long)n * n, count, eps_s, r.sums, st, r.lmax));
   if (scaling == SHP_SCALE_FROBENIUS) {
     GEMM_TRY(launch_sqrt_scale(r.sums, nullptr, scale_out, count, st));
     return SHP_OK;
@@ -253,7 +255,8 @@ EpiOut final_out(float* X, int n) { return plain_out(X, n, (long long)n * n); }
 // calls ("DASH", §3 Newton-DB).
 shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec pr, RootBufs& r,
                    const float* scale, float* X, int* status, cudaStream_t st) {
-  GEMM_TRY(launch_to_planes(A, n, (long long)n * n, nullptr, count, n, n, 1.f, eps, 0.f, scale, r.Y[0], pr, st));
+  GEMM_TRY(launch_to_planes(A, n, (long long)n * n, nullptr, count, n, n, 1.f, eps, 0.f, scale, r.Y[0], pr, st,
+                            r.lmax));
   int cur = 0;
   for (int call = 0; call < 2; ++call) {
     // iteration 1 (Z_0 = I): Y_1 = Y_0 (3I - Y_0)/2 = 1.5 Y_0 - 0.5 Y_0^2, Z_1 = 1.5 I - 0.5 Y_0
@@ -317,14 +320,16 @@ shp_status run_cn(const float* A, int count, int n, float eps, int iters, Prec p
   Planes* Xp = r.Y;
   Planes* Mp = r.Z;
   const long long bs = (long long)n * n;
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 1.f, eps, 0.f, scale, Mp[0], pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 1.f, eps, 0.f, scale, Mp[0], pr, st, r.lmax));
   // T_0 = 1.25 I - 0.25 M_0 = (-0.25/s) L + (1.25 - 0.25 eps/s) I ; X_1 = X_0 T_0 = T_0
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, r.T, pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, r.T, pr, st,
+                            r.lmax));
   if (iters == 1) {
     GEMM_TRY(launch_scaled_copy(r.T, n, count, scale, X, status, st));
     return SHP_OK;
   }
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, Xp[0], pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, Xp[0], pr, st,
+                            r.lmax));
   int cx = 0, cm = 0;
   for (int it = 1; it <= iters; ++it) {
     const bool last = it == iters;
@@ -373,21 +378,23 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   Planes* Bk2 = &r.Z[1];
   Planes* Bk = &r.T;
   if (degree == 0) {
-    GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[0], nullptr, *Bk2, pr, st));
+    GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[0], nullptr, *Bk2, pr, st,
+                              r.lmax));
     GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, X, status, st));
     return SHP_OK;
   }
   if (degree == 1) {  // c0 I + c1 S = (2 c1/s) L + (c0 - c1) I
     GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, (float)(2 * c[1]), 0.f, (float)(c[0] - c[1]), scale,
-                              *Bk2, pr, st));
+                              *Bk2, pr, st, r.lmax));
     GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, X, status, st));
     return SHP_OK;
   }
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 2.f, 0.f, -1.f, scale, S, pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 2.f, 0.f, -1.f, scale, S, pr, st, r.lmax));
   // B_d = c_d I ; B_{d-1} = c_{d-1} I + 2 c_d S = (4 c_d / s) L + (c_{d-1} - 2 c_d) I
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[degree], nullptr, *Bk2, pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[degree], nullptr, *Bk2, pr, st,
+                            r.lmax));
   GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, (float)(4 * c[degree]), 0.f,
-                            (float)(c[degree - 1] - 2 * c[degree]), scale, *Bk1, pr, st));
+                            (float)(c[degree - 1] - 2 * c[degree]), scale, *Bk1, pr, st, r.lmax));
   for (int k = degree - 2; k >= 1; --k) {
     // B_k = c_k I + 2 S B_{k+1} - B_{k+2}; three buffers, so that no launch
     // writes a matrix it reads

@@ -112,15 +112,17 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
 
 // dst = (alpha/s_b) * src + (eps/s_b + delta) * I, written in the planes of
 // `dst` for precision `prec`.  src: count matrices rows x cols (ld, bs),
-// optional batch index map; s_b = scale[b] or 1.  For FP32 planes a first
-// pass finds max |dst| per matrix, which fixes the scale exponent.
+// optional batch index map; s_b = scale[b] or 1.  For FP32 planes the scale
+// exponent comes from max |dst| per matrix: found by a first pass, or bounded
+// by |alpha/s_b| src_amax[src b] + |eps/s_b + delta| when src_amax is given.
 cudaError_t launch_to_planes(const float* src, int src_ld, long long src_bs, const int* src_idx, int count,
                              int rows, int cols, float alpha, float eps, float delta, const float* scale,
-                             const Planes& dst, Prec prec, cudaStream_t stream);
+                             const Planes& dst, Prec prec, cudaStream_t stream, const float* src_amax = nullptr);
 
-// sums[b] += sum_ij (L_ij + eps*delta_ij)^2 for each matrix (double atomics).
+// sums[b] = sum_ij (L_ij + eps*delta_ij)^2 for each matrix (double atomics)
+// and, when amax is given, amax[b] = max_ij |L_ij|.  n, ld, bs multiples of 4.
 cudaError_t launch_frob_sumsq(const float* L, int n, int ld, long long bs, int count, float eps, double* sums,
-                              cudaStream_t stream);
+                              cudaStream_t stream, float* amax = nullptr);
 // scale[b] = sqrt(sums[b]) * factor[b] (factor may be null)
 cudaError_t launch_sqrt_scale(const double* sums, const float* factor, float* scale, int count,
                               cudaStream_t stream);

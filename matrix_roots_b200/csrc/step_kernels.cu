@@ -87,15 +87,37 @@ __global__ void graft_pass1_kernel(const int* __restrict__ blocks, int block0, L
   float* V = la.v[li];
   const long long total = (long long)rows * cols;
   float acc = 0.f;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(e / cols), c = (int)(e - (long long)r * cols);
-    const long long off = (long long)(r0 + r) * lc + c0 + c;
-    float dm = 0.f, dv = 0.f;
-    float* pm = M ? M + off : &dm;
-    float* pv = V ? V + off : &dv;
-    const float g = graft_value(s.kind, G[off], pm, pv, s);
-    acc = fmaf(g, g, acc);
+  if (((cols | c0 | lc) & 3) == 0) {
+    // float4 quads of a row; 32-bit indices (a block holds < 2^31 elements)
+    const int q = cols >> 2, tq = rows * q;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < tq; e += gridDim.x * blockDim.x) {
+      const int r = e / q, c = (e - r * q) * 4;
+      const long long off = (long long)(r0 + r) * lc + c0 + c;
+      const float4 g4 = *reinterpret_cast<const float4*>(G + off);
+      float4 m4 = M ? *reinterpret_cast<const float4*>(M + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v4 = V ? *reinterpret_cast<const float4*>(V + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float a = graft_value(s.kind, g4.x, &m4.x, &v4.x, s);
+      const float b = graft_value(s.kind, g4.y, &m4.y, &v4.y, s);
+      const float c2 = graft_value(s.kind, g4.z, &m4.z, &v4.z, s);
+      const float d = graft_value(s.kind, g4.w, &m4.w, &v4.w, s);
+      if (M && s.kind == GRAFT_ADAM) *reinterpret_cast<float4*>(M + off) = m4;
+      if (V && s.kind != GRAFT_SGD) *reinterpret_cast<float4*>(V + off) = v4;
+      acc = fmaf(a, a, acc);
+      acc = fmaf(b, b, acc);
+      acc = fmaf(c2, c2, acc);
+      acc = fmaf(d, d, acc);
+    }
+  } else {
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+      const int r = (int)(e / cols), c = (int)(e - (long long)r * cols);
+      const long long off = (long long)(r0 + r) * lc + c0 + c;
+      float dm = 0.f, dv = 0.f;
+      float* pm = M ? M + off : &dm;
+      float* pv = V ? V + off : &dv;
+      const float g = graft_value(s.kind, G[off], pm, pv, s);
+      acc = fmaf(g, g, acc);
+    }
   }
   const float tot = block_sum(acc, red);
   if (threadIdx.x == 0) atomicAdd(gsum + bid, (double)tot);
@@ -136,11 +158,26 @@ __global__ void graft_pass2_kernel(const int* __restrict__ blocks, const int* __
   float* W = la.W[li];
   const float* D = dptr.ptr[gb] + (long long)gi * rows * cols;
   const long long total = (long long)rows * cols;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(e / cols), c = (int)(e - (long long)r * cols);
-    const long long off = (long long)(r0 + r) * lc + c0 + c;
-    W[off] = keep * W[off] - step * D[(long long)r * cols + c];
+  if (((cols | c0 | lc) & 3) == 0) {
+    const int q = cols >> 2, tq = rows * q;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < tq; e += gridDim.x * blockDim.x) {
+      const int r = e / q, c = (e - r * q) * 4;
+      const long long off = (long long)(r0 + r) * lc + c0 + c;
+      float4 w = *reinterpret_cast<const float4*>(W + off);
+      const float4 d = *reinterpret_cast<const float4*>(D + (long long)r * cols + c);
+      w.x = keep * w.x - step * d.x;
+      w.y = keep * w.y - step * d.y;
+      w.z = keep * w.z - step * d.z;
+      w.w = keep * w.w - step * d.w;
+      *reinterpret_cast<float4*>(W + off) = w;
+    }
+  } else {
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+      const int r = (int)(e / cols), c = (int)(e - (long long)r * cols);
+      const long long off = (long long)(r0 + r) * lc + c0 + c;
+      W[off] = keep * W[off] - step * D[(long long)r * cols + c];
+    }
   }
 }
 

@@ -72,6 +72,9 @@ def make_grads(shapes, seed, kind="transformer"):
     return W.transformer_grads(shapes, seed=seed)
 
 
+GEMM_DRAM_BYTES_PER_LAUNCH = 3459.7e6
+
+
 def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters):
     """Algorithmic FLOPs of one shampoo_inv_root call (2 n^3 per matmul)."""
     if method == "ndb":
@@ -338,8 +341,12 @@ def run_ours(args, cfg):
     passes = {"fp32": 3.0, "tf32": 2.0, "fp16": 1.0, "bf16": 1.0}[args.dtype]
     peak = peaks["bf16_sust"] / passes
     achieved = flops / (root_ms / 1000.0) / 1e12
+    # DRAM bytes per launch of the FP32 GEMM on this workload, from the ncu
+    # launch list in profiles/launches_transformer_step.txt (mean over the
+    # 121 captured launches); other workloads / dtypes were not captured
+    traffic = GEMM_DRAM_BYTES_PER_LAUNCH if (args.config == "transformer" and args.dtype == "fp32") else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None,
+                "traffic": traffic, "traffic_unit": "DRAM bytes per launch (read + write)",
                 "kernel": "gemm_kernel (all launches inside shampoo_inv_root)",
                 "peak_note": f"{peaks['source']} sustained bf16 rate / {passes:g} (fp16-rate MMA work per "
                              f"algorithmic flop, {args.dtype})",

@@ -375,32 +375,35 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
   using C = Cfg<KIND, NPASS, BN>;
   using KT = KindTraits<KIND>;
   constexpr int S = C::STAGES;
-  constexpr int NB = C::NBUF;
   constexpr int BKE = C::BKE;
-  constexpr int DR = C::DRAIN;
   constexpr int KS = BKE / KT::KINST;  // MMA slices per K-block (4)
+  // TMEM: NBUF slots of BN columns, used in groups: FP32 mode fills a pair
+  // of slots per K-block (two 32-deep halves), the one-pass modes one slot
+  // per DRAIN K-blocks
+  constexpr int SPG = (NPASS == 3) ? 2 : 1;
+  constexpr int NG = C::NBUF / SPG;
+  constexpr int KPG = (NPASS == 3) ? 1 : C::DRAIN;
+  // one tcgen05.commit per K-block, onto kdone[k % Q]: the producer waits on
+  // it to reuse the K-block's stage, the draining warps to read its slots;
+  // neither lags the issuer by Q K-blocks or more (S <= 8, NG * KPG <= 16)
+  constexpr int Q = 32;
+  static_assert(S < Q && NG * KPG < Q, "completion ring too short");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NB + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S + Q + NG + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * S;
-  const uint32_t tfull0 = empty0 + 8 * S;    // [NB] slot written by the MMA
-  const uint32_t tempty0 = tfull0 + 8 * NB;  // [NB] slot drained by all 8 draining warps
-  const uint32_t done_bar = tempty0 + 8 * NB;  // last MMAs of this CTA complete
+  const uint32_t full0 = smem_u32(bars);       // [S] stage loaded (TMA complete_tx)
+  const uint32_t kdone0 = full0 + 8 * S;       // [Q] MMAs of a K-block complete
+  const uint32_t tempty0 = kdone0 + 8 * Q;     // [NG] slot group drained by all 8 draining warps
+  const uint32_t done_bar = tempty0 + 8 * NG;  // last MMAs of this CTA complete
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    for (int j = 0; j < NB; ++j) {
-      mbar_init(tfull0 + 8 * j, 1);
-      mbar_init(tempty0 + 8 * j, 8);  // one arrival per draining warp
-    }
+    for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 1);
+    for (int j = 0; j < Q; ++j) mbar_init(kdone0 + 8 * j, 1);
+    for (int j = 0; j < NG; ++j) mbar_init(tempty0 + 8 * j, 8);  // one arrival per draining warp
     mbar_init(done_bar, 1);
     // skip all tiles once any CTA has given up on a barrier
     *abort_flag = (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) ? 1 : 0;
@@ -420,7 +423,7 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
     // ---- TMA producer ----
     if (lane == 0) {
       Ring st;
-      long long issued = 0;
+      uint32_t gk = 0;  // K-blocks loaded so far
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
@@ -431,10 +434,14 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         const int a_mn = g.a_mn, b_mn = g.b_mn;
         const int a4 = p.a4d[x.grp], b4 = p.b4d[x.grp];
         bool ok = true;
-        for (int kb = 0, k0 = 0; kb < x.nk; ++kb, k0 += BKE) {
-          if (!mbar_wait(empty0 + 8 * st.i, st.ph ^ 1)) {
-            ok = false;
-            break;
+        for (int kb = 0, k0 = 0; kb < x.nk; ++kb, k0 += BKE, ++gk) {
+          // the stage was last read by K-block gk - S
+          if (gk >= (uint32_t)S) {
+            const uint32_t o = gk - S;
+            if (!mbar_wait(kdone0 + 8 * (o % Q), (o / Q) & 1)) {
+              ok = false;
+              break;
+            }
           }
           const uint32_t fb = full0 + 8 * st.i;
           mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
@@ -462,7 +469,6 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
             }
           }
           st.template next<S>();
-          ++issued;
         }
         if (!ok) {
           *abort_flag = 1;
@@ -472,7 +478,8 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       // after an abort, loads may still be landing in stages nobody waited
       // for: let the latest load of every stage finish before the shared
       // memory is given up (immediate when all were consumed)
-      for (long long n = issued - 1; n >= 0 && n >= issued - S; --n) mbar_wait(full0 + 8 * (n % S), (n / S) & 1);
+      for (long long n = (long long)gk - 1; n >= 0 && n >= (long long)gk - S; --n)
+        mbar_wait(full0 + 8 * (n % S), (n / S) & 1);
     }
   } else if (warp == 8) {
     // ---- MMA issuer ----
@@ -481,8 +488,9 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       constexpr uint32_t KSTEP_MN = KT::KINST * 128;    // KINST rows of 128 bytes
       constexpr uint32_t LBO_MN = BKE * 128;            // one TMA box along M/N
       const uint32_t smem0 = smem_u32(smem);
-      Ring st, sl;
-      int in_slot = 0;  // K-blocks already accumulated in the current slot
+      Ring st, gr;
+      uint32_t gk = 0;  // K-blocks issued so far
+      int in_group = 0;  // K-blocks already accumulated in the current slot group
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
@@ -497,25 +505,22 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         const uint64_t a_step = (g.a_mn ? KSTEP_MN : KSTEP_K) >> 4;
         const uint64_t b_step = (g.b_mn ? KSTEP_MN : KSTEP_K) >> 4;
         bool ok = true;
-        for (int kb = 0; kb < x.nk && ok; ++kb) {
-          if (!mbar_wait(full0 + 8 * st.i, st.ph)) {
+        for (int kb = 0; kb < x.nk; ++kb, ++gk) {
+          if (!mbar_wait(full0 + 8 * st.i, st.ph) ||
+              (in_group == 0 && !mbar_wait(tempty0 + 8 * gr.i, gr.ph ^ 1))) {
             ok = false;
             break;
           }
+          tc_fence_after();
           const uint64_t so = (uint64_t)(st.i * (C::STAGE_BYTES >> 4));
           const uint64_t ad = a0 + so, bd = b0 + so;
           if constexpr (NPASS == 3) {
-            // two TMEM slots per K-block, 32 K each: in each, the correction
-            // products lo*hi and hi*lo first (in units of 2^-11), then hi*hi,
-            // the first of which scales the slot by 2^-11
+            // two slots, 32 K each: in each, the correction products lo*hi
+            // and hi*lo first (in units of 2^-11), then hi*hi, the first of
+            // which scales the slot by 2^-11
 #pragma unroll
-            for (int hs = 0; hs < KS / 2; ++hs) {
-              if (!mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t d = tmem + sl.i * BN;
+            for (int hs = 0; hs < 2; ++hs) {
+              const uint32_t d = tmem + (gr.i * 2 + hs) * BN;
 #pragma unroll
               for (int ks = 2 * hs; ks < 2 * hs + 2; ++ks) {
                 mma<KIND>(d, ad + (C::A_TILE >> 4) + ks * a_step, bd + ks * b_step, idesc, ks > 2 * hs ? 1u : 0u);
@@ -523,29 +528,18 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
               }
               mma_f16_scale11(d, ad + 2 * hs * a_step, bd + 2 * hs * b_step, idesc);
               mma<KIND>(d, ad + (2 * hs + 1) * a_step, bd + (2 * hs + 1) * b_step, idesc, 1u);
-              tc_commit(tfull0 + 8 * sl.i);
-              sl.template next<NB>();
             }
-            if (!ok) break;
-            tc_commit(empty0 + 8 * st.i);
-            st.template next<S>();
           } else {
-            if (in_slot == 0 && !mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t d = tmem + sl.i * BN;
+            const uint32_t d = tmem + gr.i * BN;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks)
-              mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, (in_slot | ks) ? 1u : 0u);
-            tc_commit(empty0 + 8 * st.i);
-            st.template next<S>();
-            if (++in_slot == DR || kb == x.nk - 1) {
-              tc_commit(tfull0 + 8 * sl.i);
-              sl.template next<NB>();
-              in_slot = 0;
-            }
+              mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, (in_group | ks) ? 1u : 0u);
+          }
+          tc_commit(kdone0 + 8 * (gk % Q));
+          st.template next<S>();
+          if (++in_group == KPG || kb == x.nk - 1) {
+            gr.template next<NG>();
+            in_group = 0;
           }
         }
         if (!ok) {
@@ -562,7 +556,8 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
     constexpr int HC = BN / 2;
     const int h = warp >> 2;
     const int q = warp & 3;
-    Ring sl;
+    Ring gr;
+    uint32_t gkb = 0;  // K-blocks of the tiles before this one
     float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + warp * 1024;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
@@ -571,26 +566,31 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
 #pragma unroll
       for (int i = 0; i < HC; ++i) acc[i] = 0.f;
       bool ok = true;
-      const int nslots = NPASS == 3 ? x.nk * (KS / 2) : (x.nk + DR - 1) / DR;
-      for (int u = 0; u < nslots; ++u) {
-        ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * sl.i, sl.ph));
+      for (int k0 = 0; k0 < x.nk; k0 += KPG) {
+        // the group is complete once its last K-block's MMAs are
+        const uint32_t last = gkb + (uint32_t)((k0 + KPG < x.nk ? k0 + KPG : x.nk) - 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(kdone0 + 8 * (last % Q), (last / Q) & 1));
         if (!ok) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        uint32_t r[HC];
-        const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(sl.i * BN + h * HC);
 #pragma unroll
-        for (int c = 0; c < HC; c += 32) tmem_ld32_nowait(base + c, r + c);
-        tmem_wait_ld();
+        for (int sj = 0; sj < SPG; ++sj) {
+          uint32_t r[HC];
+          const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((gr.i * SPG + sj) * BN + h * HC);
 #pragma unroll
-        for (int i = 0; i < HC; ++i) acc[i] += __uint_as_float(r[i]);
+          for (int c = 0; c < HC; c += 32) tmem_ld32_nowait(base + c, r + c);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < HC; ++i) acc[i] += __uint_as_float(r[i]);
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty0 + 8 * sl.i);
-        sl.template next<NB>();
+        if (lane == 0) mbar_arrive(tempty0 + 8 * gr.i);
+        gr.template next<NG>();
       }
+      gkb += (uint32_t)x.nk;
       if (!ok) break;
       const GroupDev& g = p.g[x.grp];
       const EpiCtx ec = make_ctx(g, x.b, lane == 0);

@@ -90,14 +90,14 @@ struct Cfg {
   static constexpr int A_TILE = 128 * 128;
   static constexpr int B_TILE = BN * 128;
   static constexpr int STAGE_BYTES = NPL * (A_TILE + B_TILE);
-  static constexpr int NBUF = 4;
+  static constexpr int NBUF = 3;  // accumulation slots; a fourth block of BN columns is the epilogue handoff
   // K-blocks accumulated in one TMEM slot before it is drained in the
   // one-pass modes, whose operand rounding (2^-11) dwarfs the accumulation
   // error; FP32 mode instead drains every half K-block (32 K), for accuracy
   static constexpr int DRAIN = (NPASS == 3) ? 1 : 4;
-  static constexpr int TCOLS = NBUF * BN;
-  static constexpr int THREADS = 320;
-  static constexpr int STAGE_OUT = 8 * 32 * 32 * 4;  // 32x32 transpose buffer per draining warp
+  static constexpr int TCOLS = 4 * BN;
+  static constexpr int THREADS = 448;
+  static constexpr int STAGE_OUT = 4 * 32 * 32 * 4;  // 32x32 transpose buffer per epilogue warp
   static constexpr int RESERVED = 1024 + 512 + STAGE_OUT;
   static constexpr int STAGES_RAW = (227 * 1024 - RESERVED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
@@ -286,13 +286,11 @@ __device__ __forceinline__ uint2 pack_half4(__half a, __half b, __half c, __half
 __device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) {
   if (o.f32) *reinterpret_cast<float4*>(o.f32 + off) = v;
   if (o.h16lo) {
-    __half h0, h1, h2, h3, l0, l1, l2, l3;
-    split16(v.x * o.sc, h0, l0);
-    split16(v.y * o.sc, h1, l1);
-    split16(v.z * o.sc, h2, l2);
-    split16(v.w * o.sc, h3, l3);
-    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) = pack_half4(h0, h1, h2, h3);
-    *reinterpret_cast<uint2*>(o.h16lo + off) = pack_half4(l0, l1, l2, l3);
+    __half2 h01, h23, l01, l23;
+    split16x2(v.x * o.sc, v.y * o.sc, h01, l01);
+    split16x2(v.z * o.sc, v.w * o.sc, h23, l23);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(o.h16) + off) = make_uint2(h2bits(h01), h2bits(h23));
+    *reinterpret_cast<uint2*>(o.h16lo + off) = make_uint2(h2bits(l01), h2bits(l23));
   } else if (o.h16) {
     if (o.bf) {
       __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
@@ -309,6 +307,7 @@ __device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) 
 
 __device__ __forceinline__ float max4(float4 v) { return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))); }
 
+template <bool NEED_C, bool HAS_X>
 __device__ __forceinline__ void epilogue_block4(const GroupDev& g, const EpiCtx& x, int row0, int col0,
                                                 const float4* stage, int lane, float& ss, int& bad, float& mo,
                                                 float& mx) {
@@ -316,34 +315,45 @@ __device__ __forceinline__ void epilogue_block4(const GroupDev& g, const EpiCtx&
   const int col = col0 + 4 * cq;
   if (col >= g.N) return;
   const OutPtrs O = out_ptrs(g.O, x.ob, row0, col, x.scO);
-  const OutPtrs X = x.has_x ? out_ptrs(g.X, x.ob, row0, col, x.scX) : O;
-  const float* cf = x.need_c ? g.C.f32 + (long long)x.ob * g.C.bs + (long long)row0 * g.C.ld + col : nullptr;
+  const OutPtrs X = HAS_X ? out_ptrs(g.X, x.ob, row0, col, x.scX) : O;
+  const float* cf = NEED_C ? g.C.f32 + (long long)x.ob * g.C.bs + (long long)row0 * g.C.ld + col : nullptr;
   const long long cld = g.C.ld;
   const int rmax = g.M - row0 < 32 ? g.M - row0 : 32;
-#pragma unroll 2
+#pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int r = it * 4 + (lane >> 3);
     if (r >= rmax) continue;
     const float4 a = stage[r * 8 + (cq ^ (r & 7))];
     float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (x.need_c) c = *reinterpret_cast<const float4*>(cf + r * cld);
+    if (NEED_C) c = *reinterpret_cast<const float4*>(cf + r * cld);
     const int e = row0 + r - col;  // component on the diagonal, if 0..3
     const float d0 = e == 0 ? 1.f : 0.f, d1 = e == 1 ? 1.f : 0.f, d2 = e == 2 ? 1.f : 0.f, d3 = e == 3 ? 1.f : 0.f;
     float4 q;
-    q.x = x.alpha * a.x + x.beta * c.x + x.gamma * d0;
-    q.y = x.alpha * a.y + x.beta * c.y + x.gamma * d1;
-    q.z = x.alpha * a.z + x.beta * c.z + x.gamma * d2;
-    q.w = x.alpha * a.w + x.beta * c.w + x.gamma * d3;
+    q.x = x.alpha * a.x + x.gamma * d0;
+    q.y = x.alpha * a.y + x.gamma * d1;
+    q.z = x.alpha * a.z + x.gamma * d2;
+    q.w = x.alpha * a.w + x.gamma * d3;
+    if (NEED_C) {
+      q.x += x.beta * c.x;
+      q.y += x.beta * c.y;
+      q.z += x.beta * c.z;
+      q.w += x.beta * c.w;
+    }
     const float4 v = make_float4(q.x * x.mult, q.y * x.mult, q.z * x.mult, q.w * x.mult);
     put4(O, (long long)r * O.ld, v);
     ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
     mo = fmaxf(mo, max4(v));
-    if (x.has_x) {
-      const float4 xv = make_float4(x.mult * (x.alpha2 * q.x + x.beta2 * c.x + x.gamma2 * d0),
-                                    x.mult * (x.alpha2 * q.y + x.beta2 * c.y + x.gamma2 * d1),
-                                    x.mult * (x.alpha2 * q.z + x.beta2 * c.z + x.gamma2 * d2),
-                                    x.mult * (x.alpha2 * q.w + x.beta2 * c.w + x.gamma2 * d3));
+    if (HAS_X) {
+      float4 xv = make_float4(x.alpha2 * q.x + x.gamma2 * d0, x.alpha2 * q.y + x.gamma2 * d1,
+                              x.alpha2 * q.z + x.gamma2 * d2, x.alpha2 * q.w + x.gamma2 * d3);
+      if (NEED_C) {
+        xv.x += x.beta2 * c.x;
+        xv.y += x.beta2 * c.y;
+        xv.z += x.beta2 * c.z;
+        xv.w += x.beta2 * c.w;
+      }
+      xv = make_float4(xv.x * x.mult, xv.y * x.mult, xv.z * x.mult, xv.w * x.mult);
       put4(X, (long long)r * X.ld, xv);
       mx = fmaxf(mx, max4(xv));
     }
@@ -371,39 +381,44 @@ struct Ring {
 };
 
 template <int KIND, int NPASS, int BN>
-__global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<KIND, NPASS, BN>;
   using KT = KindTraits<KIND>;
   constexpr int S = C::STAGES;
   constexpr int BKE = C::BKE;
   constexpr int KS = BKE / KT::KINST;  // MMA slices per K-block (4)
-  // TMEM: NBUF slots of BN columns, used in groups: FP32 mode fills a pair
-  // of slots per K-block (two 32-deep halves), the one-pass modes one slot
-  // per DRAIN K-blocks
-  constexpr int SPG = (NPASS == 3) ? 2 : 1;
-  constexpr int NG = C::NBUF / SPG;
+  // TMEM: NS accumulation slots of BN columns in a ring, then the handoff
+  // block read by the epilogue warps.  FP32 mode fills two slots per K-block
+  // (two 32-deep halves), the one-pass modes one slot per DRAIN K-blocks.
+  constexpr int NS = C::NBUF;
+  constexpr int SPK = (NPASS == 3) ? 2 : 1;  // slots per drained group
   constexpr int KPG = (NPASS == 3) ? 1 : C::DRAIN;
+  constexpr uint32_t HANDOFF = NS * BN;
   // one tcgen05.commit per K-block, onto kdone[k % Q]: the producer waits on
   // it to reuse the K-block's stage, the draining warps to read its slots;
-  // neither lags the issuer by Q K-blocks or more (S <= 8, NG * KPG <= 16)
+  // neither lags the issuer by Q K-blocks or more
   constexpr int Q = 32;
-  static_assert(S < Q && NG * KPG < Q, "completion ring too short");
+  static_assert(S < Q && NS * KPG < Q, "completion ring too short");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S + Q + NG + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S + Q + NS + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t full0 = smem_u32(bars);       // [S] stage loaded (TMA complete_tx)
-  const uint32_t kdone0 = full0 + 8 * S;       // [Q] MMAs of a K-block complete
-  const uint32_t tempty0 = kdone0 + 8 * Q;     // [NG] slot group drained by all 8 draining warps
-  const uint32_t done_bar = tempty0 + 8 * NG;  // last MMAs of this CTA complete
+  const uint32_t full0 = smem_u32(bars);        // [S] stage loaded (TMA complete_tx)
+  const uint32_t kdone0 = full0 + 8 * S;        // [Q] MMAs of a K-block complete
+  const uint32_t tempty0 = kdone0 + 8 * Q;      // [NS] slot drained by all 8 draining warps
+  const uint32_t hfull = tempty0 + 8 * NS;      // handoff written by the 8 draining warps
+  const uint32_t hempty = hfull + 8;            // handoff read by the 4 epilogue warps
+  const uint32_t done_bar = hempty + 8;         // last MMAs of this CTA complete
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) mbar_init(full0 + 8 * s, 1);
     for (int j = 0; j < Q; ++j) mbar_init(kdone0 + 8 * j, 1);
-    for (int j = 0; j < NG; ++j) mbar_init(tempty0 + 8 * j, 8);  // one arrival per draining warp
+    for (int j = 0; j < NS; ++j) mbar_init(tempty0 + 8 * j, 8);  // one arrival per draining warp
+    mbar_init(hfull, 8);
+    mbar_init(hempty, 4);
     mbar_init(done_bar, 1);
     // skip all tiles once any CTA has given up on a barrier
     *abort_flag = (*reinterpret_cast<volatile int*>(&shp_dev_error) != 0) ? 1 : 0;
@@ -488,9 +503,9 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       constexpr uint32_t KSTEP_MN = KT::KINST * 128;    // KINST rows of 128 bytes
       constexpr uint32_t LBO_MN = BKE * 128;            // one TMA box along M/N
       const uint32_t smem0 = smem_u32(smem);
-      Ring st, gr;
+      Ring st, sl;
       uint32_t gk = 0;  // K-blocks issued so far
-      int in_group = 0;  // K-blocks already accumulated in the current slot group
+      int in_group = 0;  // K-blocks already accumulated in the current slot (one-pass modes)
       for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
         const Tile x = decode_tile(p, t, BN, BKE);
         const GroupDev& g = p.g[x.grp];
@@ -505,13 +520,11 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         const uint64_t a_step = (g.a_mn ? KSTEP_MN : KSTEP_K) >> 4;
         const uint64_t b_step = (g.b_mn ? KSTEP_MN : KSTEP_K) >> 4;
         bool ok = true;
-        for (int kb = 0; kb < x.nk; ++kb, ++gk) {
-          if (!mbar_wait(full0 + 8 * st.i, st.ph) ||
-              (in_group == 0 && !mbar_wait(tempty0 + 8 * gr.i, gr.ph ^ 1))) {
+        for (int kb = 0; kb < x.nk && ok; ++kb, ++gk) {
+          if (!mbar_wait(full0 + 8 * st.i, st.ph)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint64_t so = (uint64_t)(st.i * (C::STAGE_BYTES >> 4));
           const uint64_t ad = a0 + so, bd = b0 + so;
           if constexpr (NPASS == 3) {
@@ -520,7 +533,12 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
             // which scales the slot by 2^-11
 #pragma unroll
             for (int hs = 0; hs < 2; ++hs) {
-              const uint32_t d = tmem + (gr.i * 2 + hs) * BN;
+              if (!mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t d = tmem + sl.i * BN;
 #pragma unroll
               for (int ks = 2 * hs; ks < 2 * hs + 2; ++ks) {
                 mma<KIND>(d, ad + (C::A_TILE >> 4) + ks * a_step, bd + ks * b_step, idesc, ks > 2 * hs ? 1u : 0u);
@@ -528,19 +546,26 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
               }
               mma_f16_scale11(d, ad + 2 * hs * a_step, bd + 2 * hs * b_step, idesc);
               mma<KIND>(d, ad + (2 * hs + 1) * a_step, bd + (2 * hs + 1) * b_step, idesc, 1u);
+              sl.template next<NS>();
             }
+            if (!ok) break;
           } else {
-            const uint32_t d = tmem + gr.i * BN;
+            if (in_group == 0 && !mbar_wait(tempty0 + 8 * sl.i, sl.ph ^ 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + sl.i * BN;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks)
               mma<KIND>(d, ad + ks * a_step, bd + ks * b_step, idesc, (in_group | ks) ? 1u : 0u);
+            if (++in_group == KPG || kb == x.nk - 1) {
+              sl.template next<NS>();
+              in_group = 0;
+            }
           }
           tc_commit(kdone0 + 8 * (gk % Q));
           st.template next<S>();
-          if (++in_group == KPG || kb == x.nk - 1) {
-            gr.template next<NG>();
-            in_group = 0;
-          }
         }
         if (!ok) {
           *abort_flag = 1;
@@ -551,14 +576,14 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
       tc_commit(done_bar);
       mbar_wait(done_bar, 0);
     }
-  } else {
-    // ---- draining warps + epilogue ----
+  } else if (warp < 8) {
+    // ---- draining warps: TMEM slots -> fp32 registers -> handoff ----
     constexpr int HC = BN / 2;
     const int h = warp >> 2;
     const int q = warp & 3;
-    Ring gr;
+    const uint32_t lanes = (uint32_t)(q * 32) << 16;
+    Ring sl, ho;
     uint32_t gkb = 0;  // K-blocks of the tiles before this one
-    float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + warp * 1024;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       if (*abort_flag) break;
       const Tile x = decode_tile(p, t, BN, BKE);
@@ -570,53 +595,101 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         // the group is complete once its last K-block's MMAs are
         const uint32_t last = gkb + (uint32_t)((k0 + KPG < x.nk ? k0 + KPG : x.nk) - 1);
         ok = __all_sync(0xffffffffu, mbar_wait(kdone0 + 8 * (last % Q), (last / Q) & 1));
-        if (!ok) {
-          *abort_flag = 1;
-          break;
-        }
+        if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int sj = 0; sj < SPG; ++sj) {
-          uint32_t r[HC];
-          const uint32_t base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((gr.i * SPG + sj) * BN + h * HC);
+        for (int sj = 0; sj < SPK; ++sj) {
+          const uint32_t base = tmem + lanes + (uint32_t)(sl.i * BN + h * HC);
 #pragma unroll
-          for (int c = 0; c < HC; c += 32) tmem_ld32_nowait(base + c, r + c);
-          tmem_wait_ld();
+          for (int c = 0; c < HC; c += 32) {
+            uint32_t r[32];
+            tmem_ld32_nowait(base + c, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < HC; ++i) acc[i] += __uint_as_float(r[i]);
+            for (int i = 0; i < 32; ++i) acc[c + i] += __uint_as_float(r[i]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty0 + 8 * sl.i);
+          sl.template next<NS>();
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty0 + 8 * gr.i);
-        gr.template next<NG>();
       }
       gkb += (uint32_t)x.nk;
-      if (!ok) break;
+      // hand the tile's sums to the epilogue warps through TMEM
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(hempty, ho.ph ^ 1));
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < HC; c += 32) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(acc[c + i]);
+        tmem_st32(tmem + lanes + HANDOFF + (uint32_t)(h * HC + c), r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(hfull);
+      ho.template next<1>();
+    }
+  } else {
+    // ---- epilogue warps 10-13: handoff -> fused epilogue -> HBM ----
+    const int q = warp & 3;  // the TMEM lane quadrant this warp may read
+    const uint32_t lanes = (uint32_t)(q * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + S * C::STAGE_BYTES + 512) + (warp - 10) * 1024;
+    Ring ho;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (*abort_flag) break;
+      const Tile x = decode_tile(p, t, BN, BKE);
       const GroupDev& g = p.g[x.grp];
       const EpiCtx ec = make_ctx(g, x.b, lane == 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(hfull, ho.ph))) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
       int bad = 0;
       float ss = 0.f, mo = 0.f, mx = 0.f;
-      if (g.vec4) {
-        float4* stage4 = reinterpret_cast<float4*>(stage);
-#pragma unroll
-        for (int ch = 0; ch < HC / 32; ++ch) {
+      const int r0 = x.m0 + q * 32;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32_nowait(tmem + lanes + HANDOFF + (uint32_t)(ch * 32), r);
+        tmem_wait_ld();
+        if (ch == BN / 32 - 1) {  // the handoff is free once its last columns are read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hempty);
+        }
+        const int c0 = x.n0 + ch * 32;
+        if (g.vec4) {
+          float4* stage4 = reinterpret_cast<float4*>(stage);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            stage4[lane * 8 + (j ^ (lane & 7))] = make_float4(acc[ch * 32 + 4 * j], acc[ch * 32 + 4 * j + 1],
-                                                              acc[ch * 32 + 4 * j + 2], acc[ch * 32 + 4 * j + 3]);
+            stage4[lane * 8 + (j ^ (lane & 7))] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
           __syncwarp();
-          epilogue_block4(g, ec, x.m0 + q * 32, x.n0 + h * HC + ch * 32, stage4, lane, ss, bad, mo, mx);
-          __syncwarp();
-        }
-      } else {
+          if (ec.need_c) {
+            if (ec.has_x)
+              epilogue_block4<true, true>(g, ec, r0, c0, stage4, lane, ss, bad, mo, mx);
+            else
+              epilogue_block4<true, false>(g, ec, r0, c0, stage4, lane, ss, bad, mo, mx);
+          } else {
+            if (ec.has_x)
+              epilogue_block4<false, true>(g, ec, r0, c0, stage4, lane, ss, bad, mo, mx);
+            else
+              epilogue_block4<false, false>(g, ec, r0, c0, stage4, lane, ss, bad, mo, mx);
+          }
+        } else {
 #pragma unroll
-        for (int ch = 0; ch < HC / 32; ++ch) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = acc[ch * 32 + c];
+          for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = __uint_as_float(r[c]);
           __syncwarp();
-          epilogue_block(g, ec, x.m0 + q * 32, x.n0 + h * HC + ch * 32 + lane, stage, lane, ss, bad, mo, mx);
-          __syncwarp();
+          epilogue_block(g, ec, r0, c0 + lane, stage, lane, ss, bad, mo, mx);
         }
+        __syncwarp();
       }
       if (g.sumsq) {
 #pragma unroll
@@ -636,6 +709,7 @@ __global__ void __launch_bounds__(320, 1) gemm_kernel(const __grid_constant__ Ge
         if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(g.X.amax) + ec.ob, __float_as_uint(mx));
       }
       if (g.status && bad) atomicOr(g.status + ec.ob, 1);
+      ho.template next<1>();
     }
   }
 

@@ -134,13 +134,11 @@ __device__ __forceinline__ uint2 half4(__half a, __half b, __half c, __half d) {
 __device__ __forceinline__ void put4(const Planes& d, long long off, float4 v, int prec, float sc) {
   if (d.f32) *reinterpret_cast<float4*>(d.f32 + off) = v;
   if (prec == P_FP32) {
-    __half h0, h1, h2, h3, l0, l1, l2, l3;
-    split16(v.x * sc, h0, l0);
-    split16(v.y * sc, h1, l1);
-    split16(v.z * sc, h2, l2);
-    split16(v.w * sc, h3, l3);
-    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(d.h16) + off) = half4(h0, h1, h2, h3);
-    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(d.h16lo) + off) = half4(l0, l1, l2, l3);
+    __half2 h01, h23, l01, l23;
+    split16x2(v.x * sc, v.y * sc, h01, l01);
+    split16x2(v.z * sc, v.w * sc, h23, l23);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(d.h16) + off) = make_uint2(h2bits(h01), h2bits(h23));
+    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(d.h16lo) + off) = make_uint2(h2bits(l01), h2bits(l23));
   } else if (prec == P_FP16 || prec == P_BF16) {
     if (d.h16_bf) {
       __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), c = __floats2bfloat162_rn(v.z, v.w);

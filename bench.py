@@ -72,7 +72,7 @@ def make_grads(shapes, seed, kind="transformer"):
     return W.transformer_grads(shapes, seed=seed)
 
 
-GEMM_DRAM_BYTES_PER_LAUNCH = 3459.7e6
+GEMM_DRAM_BYTES_PER_LAUNCH = 3744.1e6
 
 
 def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters):

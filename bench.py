@@ -401,6 +401,69 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+SPD_METHODS = [("cheb", 32, "fp32"), ("cheb", 32, "fp16"), ("ndb", 20, "fp32"), ("cn", 20, "fp16"),
+               ("cn", 20, "bf16")]
+
+
+def run_spd(args):
+    """Ill-conditioned roots: 512 SPD 256^2 matrices Q diag(lam) Q^T, lam
+    log-uniform in [1e-6, 1], eps = 1e-8, Frobenius scaling; every method and
+    precision of the workload timed as shampoo_inv_root calls on
+    device-resident inputs (CUDA events; each call streams 3-5 work stacks
+    of 128 MB, larger than L2).  value = NDB-20 FP32 matrices/s; all
+    methods under "methods"."""
+    import torch
+    from matrix_roots_b200 import binding as B
+    from matrix_roots_b200 import build
+    from matrix_roots_b200 import workloads as W
+    build.build()
+    A32, _, _ = W.spd_stack(512, 256, seed=0)
+    A = torch.from_numpy(A32).cuda()
+    count, n = A.shape[0], A.shape[1]
+    peaks = load_peaks()
+    rows = {}
+    l0 = B.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        run_spd_methods(A, count, n, args, peaks, rows)
+    launches = B.launch_count() - l0
+    ref = rows["ndb20_fp32"]
+    out = {"metric": "inverse-root throughput (ill-conditioned SPD stack)", "value": ref["matrices_per_s"],
+           "unit": "matrices/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ref["ms"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (3 fp16 passes)",
+           "data": "synthetic",
+           "config": {"workload": "spd_512x256_logunif_1e-6_1", "eps": 1e-8, "scaling": "frobenius",
+                      "l2": "workspace larger than L2 (no flush)"},
+           "roofline": {"bound": "tensor", "achieved": ref["tflops_algorithmic"],
+                        "peak": peaks["bf16_sust"] / 3.0, "unit": "TFLOP/s", "frac": ref["frac"], "traffic": None,
+                        "kernel": "gemm_kernel (NDB-20 FP32)"},
+           "methods": rows, "gpu_launches": launches, "clocks": clocks.summary()}
+    print(json.dumps(out), flush=True)
+
+
+def run_spd_methods(A, count, n, args, peaks, rows):
+    import torch
+    from matrix_roots_b200 import binding as B
+    for method, iters, dtype in SPD_METHODS:
+        ws = torch.empty(B.inv_root_workspace_bytes(count, n, method, dtype, "frobenius"), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(args.warmup):
+            B.inv_root(A, 1e-8, method, iters, dtype, "frobenius", workspace=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            B.inv_root(A, 1e-8, method, iters, dtype, "frobenius", workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        fl = root_flops(n, count, method, iters, "frobenius", 0, 0)
+        passes = {"fp32": 3.0, "tf32": 2.0, "fp16": 1.0, "bf16": 1.0}[dtype]
+        rows[f"{method}{iters}_{dtype}"] = {"ms": ms, "matrices_per_s": count / (ms / 1000.0),
+                                           "tflops_algorithmic": fl / (ms / 1000.0) / 1e12,
+                                           "frac": fl / (ms / 1000.0) / 1e12 / (peaks["bf16_sust"] / passes)}
+        del ws
+
+
 def run_root_stack(args):
     """Small fixed case of the dominant kernel for profilers: Newton-DB-20
     on `args.root_stack` factors L = G G^T of transformer gradient blocks
@@ -433,7 +496,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="transformer", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="transformer", choices=sorted(CONFIGS) + ["spd_stack"])
     ap.add_argument("--dtype", default="fp32", choices=["fp32", "tf32", "fp16", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -443,6 +506,13 @@ def main():
     args.warmup = max(args.warmup, 3)
     if args.root_stack:
         run_root_stack(args)
+        return
+    if args.config == "spd_stack":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the optimizer-step "
+                                                                  "workloads; spd_stack times inverse roots only"}))
+            return
+        run_spd(args)
         return
     cfg = CONFIGS[args.config]
     if args.impl == "reference":

@@ -1,5 +1,10 @@
 """One blocked-Shampoo optimizer step as a sequence of the five C-ABI calls.
 
+With ``precond_every`` = f > 1 the roots are recomputed only on steps 1,
+1 + f, ... and the stale roots precondition the steps between ("3D-Shampoo
+optimizer" README, Hyperparameters: preconditioning_compute_steps; DASH §1,
+roots every 10-100 steps); the statistics are updated every step.
+
 ``BlockedShampoo`` owns the device state (gradient / factor / root /
 direction stacks, graft moments and one shared workspace) and calls, in
 order: shampoo_stack_blocks, shampoo_update_stats, shampoo_inv_root (once
@@ -37,6 +42,7 @@ class ShampooConfig:
     graft_eps: float = 1e-8
     weight_decay: float = 0.0
     graft_per_block: bool = False
+    precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...; statistics every step
 
 
 class BlockedShampoo:
@@ -79,7 +85,8 @@ class BlockedShampoo:
         self.t += 1
         B.stack_blocks(self.plan, G, self.g_stacks, stream)
         B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
-        for fb, (n, _) in enumerate(self.tables["f_buckets"]):
+        fresh = (self.t - 1) % max(int(c.precond_every), 1) == 0
+        for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
             B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
                        self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,

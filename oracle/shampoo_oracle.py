@@ -42,6 +42,9 @@ R7  Multi-power-iteration: V <- normalise(A V) `iters` times, then the
     largest Rayleigh quotient v^T A v; start vectors are an input.
 R8  Grafting is layerwise by default; Adam bias-corrected with eps_g; decoupled
     weight decay W <- W - lr*rho*D - lr*wd*W; rho = 0 when ||D|| = 0.
+R9  Preconditioner frequency f: statistics every step, roots on steps
+    1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
+    Hyperparameters: preconditioning_compute_steps; [DASH] §1).
 
 Parity unpinned: the power-iteration iteration count (R7: no page fixes it),
 the step-count example of [DASH] §3 (Frobenius scaling 5 -> 15 steps).
@@ -59,7 +62,7 @@ __all__ = [
     "ndb_matrix", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
     "cn_matrix", "cn_inv_root", "cn_scalar", "cn_inv_root_replay",
     "cheb_coefficients", "clenshaw_scalar", "cheb_matrix", "cheb_inv_root", "cheb_inv_root_replay",
-    "inv_root", "precondition", "graft_update", "ShampooState", "shampoo_step",
+    "inv_root", "precondition", "graft_update", "ShampooState", "compute_roots", "shampoo_step",
     "rel_fro", "round_mantissa", "truncate_mantissa", "precision_floor",
 ]
 
@@ -585,27 +588,11 @@ class ShampooState:
         self.m = [np.zeros(s) for s in self.shapes] if graft == "adam" else [None] * len(self.shapes)
         self.v = [np.zeros(s) for s in self.shapes] if need else [None] * len(self.shapes)
         self.step = 0
+        self.roots = None  # the last computed inverse roots, per factor bucket
 
 
-def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, eps: float,
-                 method: str, iters: int, scaling: str, graft: str, lr: float,
-                 beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
-                 wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
-                 replay: bool = True, prec=None):
-    """One optimizer step over all layers; returns the new weights.
-
-    ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
-    (bucket, index), so a caller can replay with another scale.
-    """
-    plan = state.plan
-    state.step += 1
-    g_st = stack_gradients(plan, grads)
-    for b in plan["blocks"]:
-        gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
-        state.factors[lb][lix], state.factors[rb][rix] = update_stats(
-            g_st[gb][gi], state.factors[lb][lix], state.factors[rb][rix], beta2, alpha)
-    if prec is not None:  # the arithmetic model also stores the statistics in float32
-        state.factors = [f.astype(np.float32).astype(np.float64) for f in state.factors]
+def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec):
+    """Inverse fourth roots of every factor of the state (a3-a6)."""
     roots = [np.empty_like(f) for f in state.factors]
     for fb, stack in enumerate(state.factors):
         for i in range(stack.shape[0]):
@@ -619,6 +606,38 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
             if scales_out is not None:
                 scales_out[(fb, i)] = s
             roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay, prec=prec)
+    return roots
+
+
+def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, eps: float,
+                 method: str, iters: int, scaling: str, graft: str, lr: float,
+                 beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
+                 wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
+                 replay: bool = True, prec=None, precond_every: int = 1):
+    """One optimizer step over all layers; returns the new weights.
+
+    ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
+    (bucket, index), so a caller can replay with another scale.
+
+    ``precond_every`` = f: the statistics are updated every step, the inverse
+    roots only on steps 1, 1 + f, 1 + 2f, ...; the steps between reuse the
+    last roots ("3D-Shampoo optimizer" README, Hyperparameters:
+    preconditioning_compute_steps; DASH §1: roots every 10-100 steps).
+    """
+    plan = state.plan
+    state.step += 1
+    g_st = stack_gradients(plan, grads)
+    for b in plan["blocks"]:
+        gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
+        state.factors[lb][lix], state.factors[rb][rix] = update_stats(
+            g_st[gb][gi], state.factors[lb][lix], state.factors[rb][rix], beta2, alpha)
+    if prec is not None:  # the arithmetic model also stores the statistics in float32
+        state.factors = [f.astype(np.float32).astype(np.float64) for f in state.factors]
+    if state.roots is not None and (state.step - 1) % max(int(precond_every), 1) != 0:
+        roots = state.roots
+    else:
+        roots = compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec)
+        state.roots = roots
     d_st = [np.empty_like(g) for g in g_st]
     for b in plan["blocks"]:
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])

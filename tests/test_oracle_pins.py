@@ -504,3 +504,32 @@ def test_full_step_sgd_graft_length():
     b = O.shampoo_step(st3, W1, G2, beta2=1.0, alpha=1.0, eps=1e-6, method="ndb", iters=40,
                        scaling="frobenius", graft="sgd", lr=0.1)
     assert O.rel_fro(b[0], a[0]) < 1e-9
+
+
+def test_stale_roots_between_preconditioner_updates():
+    """Roots every f steps ("3D-Shampoo optimizer" README, Hyperparameters:
+    preconditioning_compute_steps).  One full-rank 8x8 block, the same G every
+    step, beta2 = 1, eps = 0, exact roots, no grafting, lr = 1: after k steps
+    L = k G G^T, so a fresh root gives D_k = k^(-1/2) D_1 exactly, while a
+    stale root (computed at step 1) gives D_k = D_1."""
+    rng = np.random.default_rng(3)
+    G = rng.standard_normal((8, 8))
+    kw = dict(beta2=1.0, alpha=1.0, eps=0.0, method="evd", iters=0, scaling="frobenius", graft="none", lr=1.0)
+
+    def deltas(f, steps):
+        st = O.ShampooState([(8, 8)], 8, "none")
+        W = [np.zeros((8, 8))]
+        out = []
+        for _ in range(steps):
+            W2 = O.shampoo_step(st, W, [G], precond_every=f, **kw)
+            out.append(W2[0] - W[0])
+            W = W2
+        return out
+
+    d1 = deltas(1, 3)
+    d2 = deltas(2, 3)
+    assert np.allclose(d1[1], d1[0] / math.sqrt(2.0), rtol=1e-9, atol=0)
+    assert np.allclose(d1[2], d1[0] / math.sqrt(3.0), rtol=1e-9, atol=0)
+    assert np.array_equal(d2[0], d1[0])
+    assert np.allclose(d2[1], d2[0], rtol=1e-12, atol=0)          # stale: roots of step 1
+    assert np.allclose(d2[2], d1[0] / math.sqrt(3.0), rtol=1e-9, atol=0)  # recomputed at step 3

@@ -237,7 +237,32 @@ def oracle_blocks_per_s(cfg, shapes, sample_blocks, seed=0):
     return nblocks / dt, dt, nblocks
 
 
+def arm_config(cfg, n_blocks, n_factors, world):
+    """The `config` object both arms print for a workload."""
+    return {"workload": cfg["workload"], "blocks_per_gpu": int(n_blocks), "factors_per_gpu": int(n_factors),
+            "method": cfg["method"], "iters": cfg["iters"], "scaling": cfg["scaling"], "graft": cfg["graft"],
+            "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"}
+
+
+def oracle_one_core(cfg, shapes):
+    """The oracle's step on one block with the BLAS pool limited to one thread."""
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(limits=1):
+            rate, dt, nb = oracle_blocks_per_s(cfg, shapes, 1)
+        return {"value": rate, "cores": 1, "sample": f"{nb} gradient block, one oracle step ({dt:.1f} s)"}
+    except Exception:  # threadpoolctl missing or no BLAS pool to limit
+        return None
+
+
 # ------------------------------------------------------------------ arms -----
+
+def plan_counts(cfg, shapes):
+    """Gradient blocks and factors of the workload on one GPU (oracle planner)."""
+    import oracle as O
+    plan = O.plan_blocks(shapes, cfg["block_size"])
+    return len(plan["blocks"]), int(sum(int(c) for _, c in plan["f_buckets"]))
+
 
 def run_reference(args, cfg):
     world, rank, local = dist_env()
@@ -258,7 +283,7 @@ def run_reference(args, cfg):
     out = {"metric": "shampoo optimizer step throughput", "value": value, "unit": "blocks/s", "impl": "reference",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": cfg["workload"], "method": cfg["method"], "iters": cfg["iters"]},
+           "config": arm_config(cfg, *plan_counts(cfg, shapes), world),
            "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": blas or cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -382,10 +407,7 @@ def run_ours(args, cfg):
                "dtype": {"fp32": "f32 (3 fp16 tensor-core passes on a scaled hi/lo split)", "tf32": "tf32",
                          "fp16": "f16", "bf16": "bf16"}[args.dtype],
                "data": "synthetic",
-               "config": {"workload": cfg["workload"], "blocks_per_gpu": n_blocks, "factors_per_gpu":
-                          int(sum(int(c) for _, c in opt.tables["f_buckets"])), "method": cfg["method"],
-                          "iters": cfg["iters"], "scaling": cfg["scaling"], "graft": cfg["graft"],
-                          "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+               "config": arm_config(cfg, n_blocks, sum(int(c) for _, c in opt.tables["f_buckets"]), world),
                "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
                "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu:
@@ -393,7 +415,7 @@ def run_ours(args, cfg):
             rate, dt, nb = oracle_blocks_per_s(cfg, shapes, args.cpu_blocks)
             out["cpu_baseline"] = {"value": rate, "unit": "blocks/s", "cores": blas or cores, "kind": "oracle",
                                    "sample": f"{nb} of the {n_blocks} gradient blocks, one oracle step "
-                                             f"({dt:.1f} s)"}
+                                             f"({dt:.1f} s)", "one_core": oracle_one_core(cfg, shapes)}
         print(json.dumps(out), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -6,23 +6,28 @@
 //
 // One persistent CTA per SM walks the 128 x BN output tiles of every matrix
 // of the stack (and of up to two problems per launch):
-//   warp 9      TMA producer: 128B-swizzled operand tiles into a STAGES-deep
-//               shared-memory ring (mbarrier complete_tx)
-//   warp 8      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 0-7   two draining warpgroups (warp w reads TMEM lanes 32*(w%4)..,
-//               group h owns columns [h*BN/2, (h+1)*BN/2) of the tile)
+//   warp 9       TMA producer: 128B-swizzled operand tiles into a STAGES-deep
+//                shared-memory ring (mbarrier complete_tx)
+//   warp 8       TMEM allocator + single-thread tcgen05.mma issuer; one
+//                tcgen05.commit per K-block onto a ring of completion barriers
+//                that the producer and the draining warps both wait on
+//   warps 0-7    draining warps (warp w reads TMEM lanes 32*(w%4).., group
+//                h = w/4 owns columns [h*BN/2, (h+1)*BN/2) of the tile)
+//   warps 10-13  epilogue warps (one per TMEM lane quadrant)
 // The tensor core's FP32 accumulation error grows with the number of
-// products chained into one accumulator, so partial products go into the
-// slots of a 4-deep TMEM ring that the draining warps add into fp32
-// registers (round to nearest) and release.  FP32 mode runs three fp16
-// passes on a scaled hi / lo split of each operand (x * 2^e = hi + lo *
-// 2^-11, e per matrix): per 32 K it issues the correction products lo*hi and
-// hi*lo into a fresh slot, then hi*hi with the input-D scale 2^-11 on the
-// first, so the corrections enter at their true weight.  Every output plane
-// set in that mode gets its exponent from a bound on its values and records
-// its max |value| for the next product.  The epilogue transposes 32x32
-// blocks through shared memory so that reads of C and writes of the output
-// planes are 128-byte (or 16-byte-per-lane) coalesced.
+// products chained into one accumulator, so partial products go into a ring
+// of three TMEM slots that the draining warps add into fp32 registers (round
+// to nearest) and release; at the end of a tile they store the sums into a
+// fourth block of TMEM, the handoff, and move on while the epilogue warps
+// read it.  FP32 mode runs three fp16 passes on a scaled hi / lo split of
+// each operand (x * 2^e = hi + lo * 2^-11, e per matrix): per 32 K it issues
+// the correction products lo*hi and hi*lo into a fresh slot, then hi*hi with
+// the input-D scale 2^-11 on the first, so the corrections enter at their
+// true weight.  Every output plane set in that mode gets its exponent from a
+// bound on its values and records its max |value| for the next product.  The
+// epilogue transposes 32x32 blocks through shared memory so that reads of C
+// and writes of the output planes are 128-byte (or 16-byte-per-lane)
+// coalesced.
 #include <atomic>
 #include <cstdio>
 #include <mutex>

@@ -42,7 +42,7 @@ R7  Multi-power-iteration: V <- normalise(A V) `iters` times, then the
     largest Rayleigh quotient v^T A v; start vectors are an input.
 R8  Grafting is layerwise by default; Adam bias-corrected with eps_g; decoupled
     weight decay W <- W - lr*rho*D - lr*wd*W; rho = 0 when ||D|| = 0.
-R9  Preconditioner frequency f: statistics every step, roots on steps
+R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
     Hyperparameters: preconditioning_compute_steps; [DASH] §1).
 

@@ -57,7 +57,9 @@ typedef int32_t shp_status;
 #define SHP_METHOD_CHEB 2 /* Chebyshev polynomial, optimised matrix Clenshaw */
 
 /* Arithmetic of the tensor-core contractions; accumulation is always FP32.
- * FP32 is emulated by three TF32 passes on hi/lo splits of both operands. */
+ * FP32 is emulated by three fp16 passes (hi*hi, lo*hi, hi*lo) on a hi/lo
+ * split of both operands scaled by a power of two per matrix
+ * (x * 2^e = hi + lo * 2^-11, about 22 significant bits). */
 #define SHP_DTYPE_FP32 0
 #define SHP_DTYPE_TF32 1
 #define SHP_DTYPE_FP16 2

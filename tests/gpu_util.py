@@ -4,11 +4,12 @@ import numpy as np
 import oracle as O
 from matrix_roots_b200 import workloads as W
 
-# Relative-Frobenius tolerances.  FP32 (3 x TF32) and TF32 roots and the
-# direction: 1e-3 (stated target).  FP16 coupled Newton: 2e-2 (stated).
-# Where the input's conditioning makes 1e-3 unreachable for IEEE float32
-# arithmetic itself, the bound is three times the error the same iteration
-# reaches in float32 numpy (oracle.fp32_error_floor), never below 1e-3.
+# Relative-Frobenius tolerances.  FP32 (three fp16 passes on a scaled hi/lo
+# split) and TF32 roots and the direction: 1e-3 (stated target).  FP16
+# coupled Newton: 2e-2 (stated).  Where the input's conditioning makes 1e-3
+# unreachable for IEEE float32 arithmetic itself, the bound is three times
+# the error the same iteration reaches in float32 numpy
+# (oracle.precision_floor), never below 1e-3.
 TOL = {"fp32": 1e-3, "tf32": 1e-3, "fp16": 2e-2, "bf16": None}
 
 

@@ -42,6 +42,10 @@ R7  Multi-power-iteration: V <- normalise(A V) `iters` times, then the
     largest Rayleigh quotient v^T A v; start vectors are an input.
 R8  Grafting is layerwise by default; Adam bias-corrected with eps_g; decoupled
     weight decay W <- W - lr*rho*D - lr*wd*W; rho = 0 when ||D|| = 0.
+R12 Root power p: p in {2, 4, 8} ([Notes] "Spreading the preconditioners":
+    the square-root power is often effective for networks made mostly of
+    linear layers); Newton-DB chains log2(p) calls, each on the previous
+    call's Y; coupled Newton and Chebyshev take p directly.
 R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
     Hyperparameters: preconditioning_compute_steps; [DASH] §1).
@@ -59,7 +63,7 @@ __all__ = [
     "BLOCK_FIELDS", "split_dim", "plan_blocks", "stack_gradients", "unstack_directions",
     "update_stats", "spd_power", "inv_root_exact",
     "frobenius_scale", "power_iteration_scale",
-    "ndb_matrix", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
+    "ndb_matrix", "ndb_calls", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
     "cn_matrix", "cn_inv_root", "cn_scalar", "cn_inv_root_replay",
     "cheb_coefficients", "clenshaw_scalar", "cheb_matrix", "cheb_inv_root", "cheb_inv_root_replay",
     "inv_root", "precondition", "graft_update", "ShampooState", "compute_roots", "shampoo_step",
@@ -283,7 +287,7 @@ def precision_floor(L, eps: float, s: float, method: str, iters: int, prec: str,
     """
     fn = {"ndb": ndb_inv_root, "cn": cn_inv_root, "cheb": cheb_inv_root}[method]
     if method == "ndb":
-        X, _ = fn(L, eps, s, iters, prec)
+        X, _ = fn(L, eps, s, iters, prec, p)
     else:
         X, _ = fn(L, eps, s, iters, p, prec)
     return rel_fro(X, inv_root(L, eps, method, iters, s, p))
@@ -318,17 +322,28 @@ def ndb_matrix(Y0, iters: int, prec=None):
     return Y, Z, mm
 
 
-def ndb_inv_root(L, eps: float, s: float, iters: int, prec=None):
-    """X ~ (L + eps I)^{-1/4} by two chained Newton-DB calls (reading R4).
+def ndb_calls(p: int) -> int:
+    """Chained Newton-DB calls for the root power p = 2^c (reading R12)."""
+    if p not in (2, 4, 8):
+        raise ValueError("Newton-DB roots: p in (2, 4, 8)")
+    return {2: 1, 4: 2, 8: 3}[p]
 
-    Call 1 on A/s gives Y ~ (A/s)^{1/2}; call 2 on that Y gives
-    Z ~ (A/s)^{-1/4}; X = s^{-1/4} Z.  Returns (X, matmuls).
+
+def ndb_inv_root(L, eps: float, s: float, iters: int, prec=None, p: int = 4):
+    """X ~ (L + eps I)^{-1/p} by chained Newton-DB calls (reading R4).
+
+    Call 1 on A/s gives Y ~ (A/s)^{1/2}, Z ~ (A/s)^{-1/2}; each further call
+    runs on the previous Y and halves the power again: two calls give
+    Z ~ (A/s)^{-1/4} (the pages' chain), three (A/s)^{-1/8}.  X = s^{-1/p} Z.
+    Returns (X, matmuls).
     """
     _, st = _model(prec)
     A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
-    Y1, _, m1 = ndb_matrix(st(A / s), iters, prec)
-    _, Z2, m2 = ndb_matrix(Y1, iters, prec)
-    return s ** -0.25 * np.asarray(Z2, np.float64), m1 + m2
+    Y, mm = st(A / s), 0
+    for _ in range(ndb_calls(p)):
+        Y, Z, m = ndb_matrix(Y, iters, prec)
+        mm += m
+    return s ** (-1.0 / p) * np.asarray(Z, np.float64), mm
 
 
 def ndb_scalar(a, iters: int):
@@ -342,7 +357,7 @@ def ndb_scalar(a, iters: int):
     return y, z
 
 
-def ndb_inv_root_replay(L, eps: float, s: float, iters: int):
+def ndb_inv_root_replay(L, eps: float, s: float, iters: int, p: int = 4):
     """Same result as ``ndb_inv_root`` via its eigenvalues.
 
     Every Newton-DB iterate is a polynomial in A, so it shares A's
@@ -351,9 +366,10 @@ def ndb_inv_root_replay(L, eps: float, s: float, iters: int):
     """
     L = np.asarray(L, dtype=np.float64)
     w, Q = np.linalg.eigh(0.5 * (L + L.T))
-    y1, _ = ndb_scalar((w + eps) / s, iters)
-    _, z2 = ndb_scalar(y1, iters)
-    return (Q * (s ** -0.25 * z2)) @ Q.T
+    y = (w + eps) / s
+    for _ in range(ndb_calls(p)):
+        y, z = ndb_scalar(y, iters)
+    return (Q * (s ** (-1.0 / p) * z)) @ Q.T
 
 
 # --------------------------------------------------------------------------
@@ -497,9 +513,9 @@ def inv_root(L, eps: float, method: str, iters: int, scale: float, p: int = 4, r
     form in arithmetic model ``prec`` when one is given)."""
     if prec is not None and method != "evd":
         fn = {"ndb": ndb_inv_root, "cn": cn_inv_root, "cheb": cheb_inv_root}[method]
-        return fn(L, eps, scale, iters, prec=prec)[0] if method == "ndb" else fn(L, eps, scale, iters, p, prec)[0]
+        return fn(L, eps, scale, iters, prec=prec, p=p)[0] if method == "ndb" else fn(L, eps, scale, iters, p, prec)[0]
     if method == "ndb":
-        return ndb_inv_root_replay(L, eps, scale, iters) if replay else ndb_inv_root(L, eps, scale, iters)[0]
+        return ndb_inv_root_replay(L, eps, scale, iters, p) if replay else ndb_inv_root(L, eps, scale, iters, p=p)[0]
     if method == "cn":
         return cn_inv_root_replay(L, eps, scale, iters, p) if replay else cn_inv_root(L, eps, scale, iters, p)[0]
     if method == "cheb":

@@ -533,3 +533,22 @@ def test_stale_roots_between_preconditioner_updates():
     assert np.array_equal(d2[0], d1[0])
     assert np.allclose(d2[1], d2[0], rtol=1e-12, atol=0)          # stale: roots of step 1
     assert np.allclose(d2[2], d1[0] / math.sqrt(3.0), rtol=1e-9, atol=0)  # recomputed at step 3
+
+
+@pytest.mark.parametrize("p", [2, 8])
+def test_ndb_root_power_chain(p):
+    """Root power p (reading R12): Newton-DB chains log2(p) calls.  On a
+    well-conditioned SPD matrix (kappa 10) 25 iterations per call converge,
+    so the result is the plain definition (L + eps I)^(-1/p) from the
+    eigendecomposition; the matrix form and the eigenvalue replay agree."""
+    rng = np.random.default_rng(30 + p)
+    Q = np.linalg.qr(rng.standard_normal((12, 12)))[0]
+    lam = np.linspace(0.1, 1.0, 12)
+    L = (Q * lam) @ Q.T
+    s = O.frobenius_scale(L, 1e-6)
+    X, mm = O.ndb_inv_root(L, 1e-6, s, 25, p=p)
+    assert mm == O.ndb_calls(p) * (1 + 3 * 24)
+    assert O.rel_fro(X, (Q * (lam + 1e-6) ** (-1.0 / p)) @ Q.T) < 1e-10
+    assert O.rel_fro(O.ndb_inv_root_replay(L, 1e-6, s, 25, p), X) < 1e-10
+    # X^p (L + eps I) = I
+    assert np.linalg.norm(np.linalg.matrix_power(X, p) @ (L + 1e-6 * np.eye(12)) - np.eye(12)) < 1e-9

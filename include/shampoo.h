@@ -167,16 +167,21 @@ SHP_API shp_status shampoo_update_stats(const shp_plan* plan, const float* const
 /* ---------------------------------------------------------------------
  * a3-a6  Damping, scaling and the inverse p-th root   ([DASH] §3, A.1-A.3)
  *
- * For each of the `count` n x n matrices L_b of the stack A:
+ * For each of the `count` n x n matrices L_b of the stack A, with the root
+ * power p in {2, 4, 8} (4: the inverse fourth root of Shampoo; 2: the
+ * square-root power the "Shampoo" notes report as often effective):
  *   NDB : s = scale of L + eps I; Y0 = (L + eps I)/s; call 1 (iters
  *         iterations of Y <- Y T, Z <- T Z, T = (3I - Z Y)/2, the first one
- *         closed-form) gives Y ~ (A/s)^(1/2); call 2 on that Y gives
- *         Z ~ (A/s)^(-1/4); X = s^(-1/4) Z.  p must be 4.
+ *         closed-form) gives Y ~ (A/s)^(1/2), Z ~ (A/s)^(-1/2); each further
+ *         call runs on the previous Y and halves the power: log2(p) calls
+ *         give Z ~ (A/s)^(-1/p); X = s^(-1/p) Z.
  *   CN  : s = scale of L + eps I; M0 = (L + eps I)/s, X0 = I;
- *         T = ((p+1)I - M)/p, X <- X T, M <- T^p M; X = s^(-1/p) X.  p = 4.
+ *         T = ((p+1)I - M)/p, X <- X T, M <- T^p M (T^p by squarings);
+ *         X = s^(-1/p) X.
  *   CHEB: s = scale of L (undamped); S = 2 L/s - I; X = s^(-1/p) sum_k c_k
  *         T_k(S) with c_k interpolating x^(-1/p) at the iters+1 Chebyshev
- *         nodes of [eps, 1 + eps] (iters = degree d, d-1 matmuls).  p = 4.
+ *         nodes of [eps, 1 + eps] (iters = degree d, d-1 matmuls).
+ * Any other p returns SHP_ERR_UNSUPPORTED.
  * scaling: SHP_SCALE_FROBENIUS (s = ||.||_F) or SHP_SCALE_POWER (s = largest
  *   Rayleigh quotient after pi_iters steps of power iteration from the
  *   pi_vectors start vectors in pi_starts, device [pi_vectors][n] float32,

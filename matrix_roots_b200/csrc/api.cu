@@ -253,25 +253,30 @@ EpiOut final_out(float* X, int n) { return plain_out(X, n, (long long)n * n); }
 
 // Newton-DB inverse fourth root: two chained coupled inverse-square-root
 // calls ("DASH", §3 Newton-DB).
-shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec pr, RootBufs& r,
+shp_status run_ndb(const float* A, int count, int n, float eps, int iters, int p, Prec pr, RootBufs& r,
                    const float* scale, float* X, int* status, cudaStream_t st) {
+  // p = 2^calls: each call halves the power, the next one starting from
+  // the previous Y with Z = I
+  const int calls = p == 2 ? 1 : (p == 4 ? 2 : 3);
   GEMM_TRY(launch_to_planes(A, n, (long long)n * n, nullptr, count, n, n, 1.f, eps, 0.f, scale, r.Y[0], pr, st,
                             r.lmax));
   int cur = 0;
-  for (int call = 0; call < 2; ++call) {
+  for (int call = 0; call < calls; ++call) {
+    const bool final_call = call == calls - 1;
     // iteration 1 (Z_0 = I): Y_1 = Y_0 (3I - Y_0)/2 = 1.5 Y_0 - 0.5 Y_0^2, Z_1 = 1.5 I - 0.5 Y_0
     // Y keeps its fp32 copy only where it will be the next call's C
     GemmGroup g = group(n, n, n, &r.Y[cur], 0, &r.Y[cur], 1);
     g.epi.alpha = -0.5f;
     g.epi.beta = 1.5f;
     g.epi.C = as_c(r.Y[cur]);
-    g.epi.O = as_out(r.Y[1 - cur], call == 0 && iters == 1);
+    g.epi.O = as_out(r.Y[1 - cur], !final_call && iters == 1);
     g.epi.X = as_out(r.Z[1 - cur], false);
     g.epi.beta2 = -0.5f;
     g.epi.gamma2 = 1.5f;
-    if (call == 1 && iters == 1) {
+    if (final_call && iters == 1) {
       g.epi.X = final_out(X, n);
       g.epi.bscale = scale;
+      g.epi.root_p = p;
       g.epi.status = status;
     }
     GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
@@ -284,19 +289,21 @@ shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec 
       gt.epi.gamma = 1.5f;
       gt.epi.O = as_out(r.T, false);
       GEMM_TRY(launch_gemm(&gt, 1, count, pr, st));
-      // Y' = Y T and Z' = T Z in one grouped launch (drop what is not needed)
+      // Y' = Y T and Z' = T Z in one grouped launch (drop what is not needed:
+      // the final call's last Y, a non-final call's last Z)
       GemmGroup gs[2];
       int ng = 0;
-      if (!(call == 1 && last)) {
+      if (!(final_call && last)) {
         gs[ng] = group(n, n, n, &r.Y[cur], 0, &r.T, 1);
-        gs[ng].epi.O = as_out(r.Y[1 - cur], call == 0 && last);
+        gs[ng].epi.O = as_out(r.Y[1 - cur], !final_call && last);
         ++ng;
       }
-      if (!(call == 0 && last)) {
+      if (!(!final_call && last)) {
         gs[ng] = group(n, n, n, &r.T, 0, &r.Z[cur], 1);
-        if (call == 1 && last) {
+        if (final_call && last) {
           gs[ng].epi.O = final_out(X, n);
           gs[ng].epi.bscale = scale;
+          gs[ng].epi.root_p = p;
           gs[ng].epi.status = status;
         } else {
           gs[ng].epi.O = as_out(r.Z[1 - cur], false);
@@ -310,26 +317,25 @@ shp_status run_ndb(const float* A, int count, int n, float eps, int iters, Prec 
   return SHP_OK;
 }
 
-// Coupled Newton for A^(-1/4) ("Shampoo" notes, coupled Newton of Guo and
-// Higham): X <- X T, M <- T^4 M, T = (5I - M)/4.
-shp_status run_cn(const float* A, int count, int n, float eps, int iters, Prec pr, RootBufs& r, const float* scale,
-                  float* X, int* status, cudaStream_t st) {
-  // Buffers: X iterates r.Y[0..1], M iterates r.Z[0..1], T = ((p+1)I - M)/p
-  // in r.T, T^2 in r.T2, T^4 in r.T4.  Products in the order X T, T T,
-  // T^2 T^2, T^4 M; the epilogue of T^4 M also writes the next T.
+// Coupled Newton for A^(-1/p) ("Shampoo" notes, coupled Newton of Guo and
+// Higham): X <- X T, M <- T^p M, T = ((p+1)I - M)/p, T^p by squarings.
+shp_status run_cn(const float* A, int count, int n, float eps, int iters, int p, Prec pr, RootBufs& r,
+                  const float* scale, float* X, int* status, cudaStream_t st) {
+  // Buffers: X iterates r.Y[0..1], M iterates r.Z[0..1], T in r.T, T^2 in
+  // r.T2, T^4 in r.T4, T^8 back in r.T2.  Products in the order X T, T T,
+  // (T^2 T^2, T^4 T^4), T^p M; the epilogue of T^p M also writes the next T.
   Planes* Xp = r.Y;
   Planes* Mp = r.Z;
   const long long bs = (long long)n * n;
+  const float ip = 1.f / (float)p, pp = (float)(p + 1) / (float)p;
   GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 1.f, eps, 0.f, scale, Mp[0], pr, st, r.lmax));
-  // T_0 = 1.25 I - 0.25 M_0 = (-0.25/s) L + (1.25 - 0.25 eps/s) I ; X_1 = X_0 T_0 = T_0
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, r.T, pr, st,
-                            r.lmax));
+  // T_0 = ((p+1) I - M_0)/p = (-1/(p s)) L + ((p+1)/p - eps/(p s)) I ; X_1 = X_0 T_0 = T_0
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -ip, -ip * eps, pp, scale, r.T, pr, st, r.lmax));
   if (iters == 1) {
-    GEMM_TRY(launch_scaled_copy(r.T, n, count, scale, X, status, st));
+    GEMM_TRY(launch_scaled_copy(r.T, n, count, scale, p, X, status, st));
     return SHP_OK;
   }
-  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -0.25f, -0.25f * eps, 1.25f, scale, Xp[0], pr, st,
-                            r.lmax));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, -ip, -ip * eps, pp, scale, Xp[0], pr, st, r.lmax));
   int cx = 0, cm = 0;
   for (int it = 1; it <= iters; ++it) {
     const bool last = it == iters;
@@ -339,6 +345,7 @@ shp_status run_cn(const float* A, int count, int n, float eps, int iters, Prec p
       if (last) {
         gs[0].epi.O = final_out(X, n);
         gs[0].epi.bscale = scale;
+        gs[0].epi.root_p = p;
         gs[0].epi.status = status;
         GEMM_TRY(launch_gemm(gs, 1, count, pr, st));
         break;
@@ -353,14 +360,24 @@ shp_status run_cn(const float* A, int count, int n, float eps, int iters, Prec p
       g2.epi.O = as_out(r.T2, false);
       GEMM_TRY(launch_gemm(&g2, 1, count, pr, st));
     }
-    GemmGroup g4 = group(n, n, n, &r.T2, 0, &r.T2, 1);  // T^4 = T^2 T^2
-    g4.epi.O = as_out(r.T4, false);
-    GEMM_TRY(launch_gemm(&g4, 1, count, pr, st));
-    GemmGroup gm = group(n, n, n, &r.T4, 0, &Mp[cm], 1);  // M' = T^4 M, next T = 1.25 I - 0.25 M'
+    Planes* Tp = &r.T2;
+    if (p >= 4) {
+      GemmGroup g4 = group(n, n, n, &r.T2, 0, &r.T2, 1);  // T^4 = T^2 T^2
+      g4.epi.O = as_out(r.T4, false);
+      GEMM_TRY(launch_gemm(&g4, 1, count, pr, st));
+      Tp = &r.T4;
+    }
+    if (p == 8) {
+      GemmGroup g8 = group(n, n, n, &r.T4, 0, &r.T4, 1);  // T^8 = T^4 T^4
+      g8.epi.O = as_out(r.T2, false);
+      GEMM_TRY(launch_gemm(&g8, 1, count, pr, st));
+      Tp = &r.T2;
+    }
+    GemmGroup gm = group(n, n, n, Tp, 0, &Mp[cm], 1);  // M' = T^p M, next T = ((p+1) I - M')/p
     gm.epi.O = as_out(Mp[1 - cm], false);
     gm.epi.X = as_out(r.T, false);
-    gm.epi.alpha2 = -0.25f;
-    gm.epi.gamma2 = 1.25f;
+    gm.epi.alpha2 = -ip;
+    gm.epi.gamma2 = pp;
     GEMM_TRY(launch_gemm(&gm, 1, count, pr, st));
     cm = 1 - cm;
   }
@@ -380,13 +397,13 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   if (degree == 0) {
     GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 0.f, 0.f, (float)c[0], nullptr, *Bk2, pr, st,
                               r.lmax));
-    GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, X, status, st));
+    GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, p, X, status, st));
     return SHP_OK;
   }
   if (degree == 1) {  // c0 I + c1 S = (2 c1/s) L + (c0 - c1) I
     GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, (float)(2 * c[1]), 0.f, (float)(c[0] - c[1]), scale,
                               *Bk2, pr, st, r.lmax));
-    GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, X, status, st));
+    GEMM_TRY(launch_scaled_copy(*Bk2, n, count, scale, p, X, status, st));
     return SHP_OK;
   }
   GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 2.f, 0.f, -1.f, scale, S, pr, st, r.lmax));
@@ -418,6 +435,7 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   g.epi.C = as_c(*Bk2);
   g.epi.O = final_out(X, n);
   g.epi.bscale = scale;
+  g.epi.root_p = p;
   g.epi.status = status;
   GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
   return SHP_OK;
@@ -723,7 +741,7 @@ static shp_status check_root_args(int32_t count, int32_t n, int32_t p, int32_t m
     return fail(SHP_ERR_INVALID_ARG, "bad scaling %d", scaling);
   if (count < 1 || count > 32767) return fail(SHP_ERR_SHAPE, "count %d outside [1, 32767]", count);
   if (n < 4 || n > SHP_MAX_N || n % 4) return fail(SHP_ERR_SHAPE, "n %d: need 4 <= n <= %d, n %% 4 == 0", n, SHP_MAX_N);
-  if (p != 4) return fail(SHP_ERR_UNSUPPORTED, "only p = 4 (inverse fourth root) is built");
+  if (p != 2 && p != 4 && p != 8) return fail(SHP_ERR_UNSUPPORTED, "root power p must be 2, 4 or 8");
   if (method == SHP_METHOD_CHEB ? (iters < 0 || iters > 1000) : (iters < 1 || iters > 1000))
     return fail(SHP_ERR_INVALID_ARG, "iters %d out of range", iters);
   if (scaling == SHP_SCALE_POWER && (pi_vectors < 1 || pi_vectors > 256 || pi_vectors % 8))
@@ -762,8 +780,8 @@ shp_status shampoo_inv_root(const float* A, int32_t count, int32_t n, float eps,
   s = compute_scale(A, count, n, eps_s, scaling, pi_vectors, pi_iters, pi_starts, r, scale_out, st);
   if (s) return s;
   const Prec pr = (Prec)dtype;
-  if (method == SHP_METHOD_NDB) return run_ndb(A, count, n, eps, iters, pr, r, scale_out, X_out, status_out, st);
-  if (method == SHP_METHOD_CN) return run_cn(A, count, n, eps, iters, pr, r, scale_out, X_out, status_out, st);
+  if (method == SHP_METHOD_NDB) return run_ndb(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
+  if (method == SHP_METHOD_CN) return run_cn(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
   return run_cheb(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
 }
 

@@ -167,7 +167,7 @@ struct EpiCtx {
 __device__ __forceinline__ EpiCtx make_ctx(const GroupDev& g, int b, bool write_exp) {
   EpiCtx c;
   c.ob = g.o_idx ? g.o_idx[b] : b;
-  c.mult = g.bscale ? rsqrtf(sqrtf(g.bscale[b])) : 1.f;
+  c.mult = g.bscale ? inv_root_mult(g.bscale[b], g.root_p) : 1.f;
   c.has_x = (g.X.f32 != nullptr) || (g.X.h16 != nullptr);
   c.need_c = (g.beta != 0.f) || (c.has_x && g.beta2 != 0.f);
   c.alpha = g.alpha;

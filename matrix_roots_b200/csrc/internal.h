@@ -54,7 +54,7 @@ struct EpiOut {
 //   x = mult_b * (alpha2 * r0 + beta2 * C + gamma2 * I)     -> X (optional)
 // with r0 = alpha * D + beta * C + gamma * I (r before the multiplier)
 //   sumsq[ob] += sum r^2 ; status[ob] |= 1 if r not finite
-// where mult_b = bscale[b]^(-1/4) when bscale != null, else 1.
+// where mult_b = bscale[b]^(-1/root_p) when bscale != null, else 1.
 struct GroupDev {
   int M = 0, N = 0, K = 0;
   int a_mn = 0, b_mn = 0;  // 1: operand stored MN-major (K rows x M/N cols)
@@ -74,6 +74,7 @@ struct GroupDev {
   float alpha2 = 0.f, beta2 = 0.f, gamma2 = 0.f;
   float* sumsq = nullptr;
   int* status = nullptr;
+  int root_p = 4;  // the multiplier is bscale^(-1/root_p)
   int vec4 = 0;  // set by the launcher: N, leading dimensions and bases allow 16-byte row segments
 };
 

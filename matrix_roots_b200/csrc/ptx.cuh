@@ -201,6 +201,13 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(uint32_t a_fmt, uint32_t b_f
          ((M >> 4) << 24);
 }
 
+// s^(-1/p) for the root powers p = 2, 4, 8 (square roots of CUDA's own).
+__device__ __forceinline__ float inv_root_mult(float s, int p) {
+  if (p == 2) return rsqrtf(s);
+  if (p == 8) return rsqrtf(sqrtf(sqrtf(s)));
+  return rsqrtf(sqrtf(s));
+}
+
 // ---- scaled fp16 hi / lo split (FP32 mode operands) ----------------------
 
 // Exponent e such that |x| <= bound implies |x * 2^e| < 2^14 (fp16 holds it

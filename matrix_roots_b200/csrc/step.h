@@ -37,7 +37,8 @@ cudaError_t launch_graft_pass1(const int* blocks, int block0, int nblk, long lon
 cudaError_t launch_graft_pass2(const int* blocks, const int* layer_first, const int* gstack_off, int block0, int nblk,
                                long long max_elems, const LayerArgs& la, const BucketArgs& d, const GraftScalars& s,
                                const double* gsum, const float* dnorm2, cudaStream_t stream);
-cudaError_t launch_scaled_copy(const Planes& P, int n, int count, const float* scale, float* out, int* status,
+// out = P * scale^(-1/p) (the root multiplier), status |= 1 where not finite.
+cudaError_t launch_scaled_copy(const Planes& P, int n, int count, const float* scale, int p, float* out, int* status,
                                cudaStream_t stream);
 
 }  // namespace shp

@@ -181,10 +181,10 @@ __global__ void graft_pass2_kernel(const int* __restrict__ blocks, const int* __
   }
 }
 
-__global__ void scaled_copy_kernel(Planes P, int n, const float* __restrict__ scale, float* __restrict__ out,
+__global__ void scaled_copy_kernel(Planes P, int n, const float* __restrict__ scale, int p, float* __restrict__ out,
                                    int* __restrict__ status) {
   const int b = blockIdx.y;
-  const float mult = rsqrtf(sqrtf(scale[b]));
+  const float mult = inv_root_mult(scale[b], p);
   const long long total = (long long)n * n;
   int bad = 0;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
@@ -233,10 +233,10 @@ cudaError_t launch_graft_pass2(const int* blocks, const int* layer_first, const 
   return cudaGetLastError();
 }
 
-cudaError_t launch_scaled_copy(const Planes& P, int n, int count, const float* scale, float* out, int* status,
+cudaError_t launch_scaled_copy(const Planes& P, int n, int count, const float* scale, int p, float* out, int* status,
                                cudaStream_t stream) {
   if (count <= 0) return cudaSuccess;
-  scaled_copy_kernel<<<dim3(grid_x((long long)n * n), count), kThreads, 0, stream>>>(P, n, scale, out, status);
+  scaled_copy_kernel<<<dim3(grid_x((long long)n * n), count), kThreads, 0, stream>>>(P, n, scale, p, out, status);
   count_launch();
   return cudaGetLastError();
 }

@@ -43,6 +43,7 @@ class ShampooConfig:
     weight_decay: float = 0.0
     graft_per_block: bool = False
     precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...; statistics every step
+    root_p: int = 4             # inverse p-th roots, p in (2, 4, 8)
 
 
 class BlockedShampoo:
@@ -87,7 +88,7 @@ class BlockedShampoo:
         B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
         fresh = (self.t - 1) % max(int(c.precond_every), 1) == 0
         for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
-            B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
+            B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, c.root_p, c.pi_vectors, c.pi_iters,
                        self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,
                        stream)

@@ -129,7 +129,8 @@ def _call_inv_root(**over):
     (dict(n=0), B.SHP_ERR_SHAPE),
     (dict(n=16384), B.SHP_ERR_SHAPE),
     (dict(count=0), B.SHP_ERR_SHAPE),
-    (dict(p=2), B.SHP_ERR_UNSUPPORTED),
+    (dict(p=3), B.SHP_ERR_UNSUPPORTED),
+    (dict(p=16), B.SHP_ERR_UNSUPPORTED),
     (dict(iters=0), B.SHP_ERR_INVALID_ARG),
     (dict(eps=float("nan")), B.SHP_ERR_INVALID_ARG),
     (dict(eps=-1.0), B.SHP_ERR_INVALID_ARG),

@@ -118,6 +118,24 @@ def test_inv_root_matches_replay(method, iters, dtype, scaling, n):
         assert rel(X[b], ref) < tol, (b, rel(X[b], ref), tol)
 
 
+@pytest.mark.parametrize("p", [2, 8])
+@pytest.mark.parametrize("method,iters", [("ndb", 14), ("cn", 14), ("cheb", 24)])
+def test_inv_root_root_powers(method, iters, p):
+    """Root power p (reading R12): Newton-DB as log2(p) chained calls,
+    coupled Newton with T^p by squarings, Chebyshev fitted to x^(-1/p);
+    FP32 against the replay with the same p, at the stated 1e-3."""
+    A = spd_stack(6, 128, cond=100.0, seed=40 + p)
+    eps = 1e-4
+    X, s, st = B.inv_root(to_dev(A), eps, method, iters, "fp32", "frobenius", p=p)
+    X, s, st = X.cpu().numpy(), s.cpu().numpy(), st.cpu().numpy()
+    assert np.all(st == 0)
+    for b in range(A.shape[0]):
+        L = A[b].astype(np.float64)
+        ref = O.inv_root(L, eps, method, iters, float(s[b]), p)
+        err = rel(X[b], ref)
+        assert err < 1e-3, (b, err)
+
+
 @pytest.mark.parametrize("dtype,tol", [("fp16", 2e-2), ("bf16", None)])
 def test_cn_half_precision(dtype, tol):
     A = spd_stack(4, 128, cond=50.0, seed=11)

@@ -304,7 +304,7 @@ def run_ours(args, cfg):
     scfg = ShampooConfig(block_size=cfg["block_size"], beta2=cfg["beta2"], alpha=cfg["alpha"], eps=cfg["eps"],
                          method=cfg["method"], iters=cfg["iters"], dtype=args.dtype, stats_dtype=args.dtype,
                          precond_dtype=args.dtype, scaling=cfg["scaling"], graft=cfg["graft"], lr=cfg["lr"],
-                         weight_decay=cfg["weight_decay"])
+                         weight_decay=cfg["weight_decay"], graph=args.graph)
     opt = BlockedShampoo(shapes, scfg, dev)
     grads_np = make_grads(shapes, seed=rank, kind=args.config)
     G = [torch.from_numpy(g).to(dev) for g in grads_np]
@@ -315,33 +315,77 @@ def run_ours(args, cfg):
     # root timing hooks: events around every inv_root call of the timed steps
     root_events = []
 
-    def step(timed):
-        c = scfg
-        ws = opt.workspace
-        opt.t += 1
+    c = scfg
+    ws = opt.workspace
+
+    def part_stats():
         B.stack_blocks(opt.plan, G, opt.g_stacks)
         B.update_stats(opt.plan, opt.g_stacks, opt.factors, c.beta2, c.alpha, c.stats_dtype, ws)
-        for fb, (n, _) in enumerate(opt.tables["f_buckets"]):
+
+    def part_root(fb):
+        n = int(opt.tables["f_buckets"][fb][0])
+        B.inv_root(opt.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
+                   opt.pi_starts.get(n), opt.roots[fb], opt.scales[fb], opt.status[fb], ws)
+
+    def part_precond():
+        B.precondition(opt.plan, opt.roots, opt.g_stacks, opt.d_stacks, opt.dnorm2, c.precond_dtype, ws)
+
+    def root_flops_of(fbs):
+        return sum(root_flops(int(opt.tables["f_buckets"][fb][0]), int(opt.tables["f_buckets"][fb][1]), c.method,
+                              c.iters, c.scaling, c.pi_vectors, c.pi_iters) for fb in fbs)
+
+    buckets = list(range(len(opt.tables["f_buckets"])))
+    graphs = {}
+
+    def run_part(name, fn):
+        if name in graphs:
+            graphs[name][0].replay()
+            opt.graph_launches += graphs[name][1]
+        else:
+            fn()
+
+    def step(timed):
+        opt.t += 1
+        run_part("stats", part_stats)
+        if graphs:  # all root calls replay as one graph
             if timed:
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            B.inv_root(opt.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, 4, c.pi_vectors, c.pi_iters,
-                       opt.pi_starts.get(int(n)), opt.roots[fb], opt.scales[fb], opt.status[fb], ws)
+            run_part("roots", None)
             if timed:
                 e1.record(stream)
-                root_events.append((e0, e1, int(n), int(opt.tables["f_buckets"][fb][1])))
-        B.precondition(opt.plan, opt.roots, opt.g_stacks, opt.d_stacks, opt.dnorm2, c.precond_dtype, ws)
+                root_events.append((e0, e1, root_flops_of(buckets)))
+        else:
+            for fb in buckets:
+                if timed:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                part_root(fb)
+                if timed:
+                    e1.record(stream)
+                    root_events.append((e0, e1, root_flops_of([fb])))
+        run_part("precond", part_precond)
         B.graft_step(opt.plan, W, G, opt.d_stacks, opt.dnorm2, opt.m, opt.v, c.graft, c.lr, c.beta1,
                      c.graft_beta2, c.graft_eps, c.weight_decay, opt.t, c.graft_per_block, ws)
 
     for _ in range(args.warmup):
+        step(False)
+    if args.graph:  # capture after the eager warm-up; the graft step stays direct (its step count changes)
+        torch.cuda.synchronize(dev)
+        for name, fn in (("stats", part_stats), ("roots", lambda: [part_root(fb) for fb in buckets]),
+                         ("precond", part_precond)):
+            gr = torch.cuda.CUDAGraph()
+            before = B.launch_count()
+            with torch.cuda.graph(gr):
+                fn()
+            graphs[name] = (gr, B.launch_count() - before)
         step(False)
     barrier(world)
     assert B.device_error() == 0, "a kernel reported a barrier timeout during warm-up"
     for s in opt.status:
         assert int(s.abs().sum()) == 0, "non-finite root during warm-up"
 
-    l0 = B.launch_count()
+    l0, g0 = B.launch_count(), opt.graph_launches
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         barrier(world)
@@ -350,16 +394,15 @@ def run_ours(args, cfg):
             step(True)
         t1.record(stream)
         barrier(world)
-    launches = B.launch_count() - l0
+    launches = B.launch_count() - l0 + (opt.graph_launches - g0)  # graph replays count their kernels
     ms_total = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms_total, world)
     ms_step = ms_max / args.steps
     value = world * n_blocks * args.steps / (ms_max / 1000.0)
 
     # roofline of the dominant kernel (the tcgen05 GEMM engine inside inv_root)
-    root_ms = sum(a.elapsed_time(b) for a, b, _, _ in root_events) / args.steps
-    flops = sum(root_flops(n, c, scfg.method, scfg.iters, scfg.scaling, scfg.pi_vectors, scfg.pi_iters)
-                for _, _, n, c in root_events) / args.steps
+    root_ms = sum(a.elapsed_time(b) for a, b, _ in root_events) / args.steps
+    flops = sum(f for _, _, f in root_events) / args.steps
     peaks = load_peaks()
     # MMA work per algorithmic flop, in units of the dense fp16/bf16 rate:
     # FP32 = three fp16 passes (hi*hi, lo*hi, hi*lo); TF32 runs at half rate
@@ -407,7 +450,8 @@ def run_ours(args, cfg):
                "dtype": {"fp32": "f32 (3 fp16 tensor-core passes on a scaled hi/lo split)", "tf32": "tf32",
                          "fp16": "f16", "bf16": "bf16"}[args.dtype],
                "data": "synthetic",
-               "config": arm_config(cfg, n_blocks, sum(int(c) for _, c in opt.tables["f_buckets"]), world),
+               "config": dict(arm_config(cfg, n_blocks, sum(int(c) for _, c in opt.tables["f_buckets"]), world),
+                              cuda_graph=bool(args.graph)),
                "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
                "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu:
@@ -522,6 +566,8 @@ def main():
     ap.add_argument("--dtype", default="fp32", choices=["fp32", "tf32", "fp16", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step's launches before the graft step as a CUDA graph")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-blocks", type=int, default=4)
     args = ap.parse_args()

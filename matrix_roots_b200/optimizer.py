@@ -44,6 +44,7 @@ class ShampooConfig:
     graft_per_block: bool = False
     precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...; statistics every step
     root_p: int = 4             # inverse p-th roots, p in (2, 4, 8)
+    graph: bool = False         # replay the launches before the graft step as a CUDA graph
 
 
 class BlockedShampoo:
@@ -78,19 +79,55 @@ class BlockedShampoo:
                for n, c in t["f_buckets"]])
         self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
         self.t = 0
+        self._graphs = {}       # (fresh roots?, gradient addresses) -> (CUDAGraph, library launches in it)
+        self.graph_launches = 0  # library kernel launches replayed from graphs so far
 
-    def step(self, W, G, stream=None) -> None:
-        """W <- W - lr * rho * D - lr * wd * W for every layer, in place."""
+    def _direction(self, G, stream, fresh: bool) -> None:
+        """Stack, statistics, roots (when fresh) and D for gradients G."""
         c = self.cfg
         ws = self.workspace
-        self.t += 1
         B.stack_blocks(self.plan, G, self.g_stacks, stream)
         B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
-        fresh = (self.t - 1) % max(int(c.precond_every), 1) == 0
         for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
             B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, c.root_p, c.pi_vectors, c.pi_iters,
                        self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,
                        stream)
+
+    def _direction_graphed(self, G, fresh: bool) -> None:
+        """The same launches replayed from a CUDA graph captured on the first
+        step that sees these gradient tensors (their addresses are part of
+        the graph: refill the same tensors every step).  The first such step
+        runs eagerly, so every kernel is set up before the capture."""
+        import torch
+        key = (fresh, tuple(int(g.data_ptr()) for g in G))
+        if key not in self._graphs:
+            if (None,) + key not in self._graphs:
+                self._graphs[(None,) + key] = None  # seen once: run eagerly
+                self._direction(G, None, fresh)
+                return
+            graph = torch.cuda.CUDAGraph()
+            before = B.launch_count()
+            torch.cuda.synchronize(self.device)
+            with torch.cuda.graph(graph):
+                self._direction(G, None, fresh)
+            self._graphs[key] = (graph, B.launch_count() - before)
+        graph, n = self._graphs[key]
+        graph.replay()
+        self.graph_launches += n
+
+    def step(self, W, G, stream=None) -> None:
+        """W <- W - lr * rho * D - lr * wd * W for every layer, in place.  With
+        ``graph`` the work before the graft step replays as a CUDA graph on the
+        current stream (the graft step's bias corrections change every step,
+        so it always launches directly)."""
+        c = self.cfg
+        ws = self.workspace
+        self.t += 1
+        fresh = (self.t - 1) % max(int(c.precond_every), 1) == 0
+        if c.graph:
+            self._direction_graphed(G, fresh)
+        else:
+            self._direction(G, stream, fresh)
         B.graft_step(self.plan, W, G, self.d_stacks, self.dnorm2, self.m, self.v, c.graft, c.lr, c.beta1,
                      c.graft_beta2, c.graft_eps, c.weight_decay, self.t, c.graft_per_block, ws, stream)

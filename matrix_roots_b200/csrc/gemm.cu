@@ -729,16 +729,17 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
 // ---- host side -------------------------------------------------------------
 
 int num_sms() {
-  static int sms[64] = {0};
+  static std::atomic<int> sms[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (!sms[dev]) {
-    int v = 0;
+  int v = sms[dev].load(std::memory_order_relaxed);
+  if (!v) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    sms[dev] = v > 0 ? v : 148;
+    if (v <= 0) v = 148;
+    sms[dev].store(v, std::memory_order_relaxed);
   }
-  return sms[dev];
+  return v;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -795,12 +796,15 @@ bool make_map_4d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int e
 template <int KIND, int NPASS, int BN>
 cudaError_t run(GemmParams& prm, cudaStream_t stream) {
   using C = Cfg<KIND, NPASS, BN>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  // the shared-memory opt-in is per device; set it once on each
+  static std::atomic<bool> attr_done[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<KIND, NPASS, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
   }
   const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
   gemm_kernel<KIND, NPASS, BN><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(prm);

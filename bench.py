@@ -304,7 +304,7 @@ def run_ours(args, cfg):
     scfg = ShampooConfig(block_size=cfg["block_size"], beta2=cfg["beta2"], alpha=cfg["alpha"], eps=cfg["eps"],
                          method=cfg["method"], iters=cfg["iters"], dtype=args.dtype, stats_dtype=args.dtype,
                          precond_dtype=args.dtype, scaling=cfg["scaling"], graft=cfg["graft"], lr=cfg["lr"],
-                         weight_decay=cfg["weight_decay"], graph=args.graph)
+                         weight_decay=cfg["weight_decay"], graph=args.graph, layerwise=args.layerwise)
     opt = BlockedShampoo(shapes, scfg, dev)
     grads_np = make_grads(shapes, seed=rank, kind=args.config)
     G = [torch.from_numpy(g).to(dev) for g in grads_np]
@@ -451,7 +451,7 @@ def run_ours(args, cfg):
                          "fp16": "f16", "bf16": "bf16"}[args.dtype],
                "data": "synthetic",
                "config": dict(arm_config(cfg, n_blocks, sum(int(c) for _, c in opt.tables["f_buckets"]), world),
-                              cuda_graph=bool(args.graph)),
+                              cuda_graph=bool(args.graph), stacking="layerwise" if args.layerwise else "gpu"),
                "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
                "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu:
@@ -566,6 +566,8 @@ def main():
     ap.add_argument("--dtype", default="fp32", choices=["fp32", "tf32", "fp16", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layerwise", action="store_true",
+                    help="stack blocks per layer (DASH-LAYERWISE) instead of across all layers")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step's launches before the graft step as a CUDA graph")
     ap.add_argument("--no-cpu", action="store_true")

@@ -123,6 +123,16 @@ SHP_API shp_status shampoo_device_error(int32_t* out);
  * On success *plan_out owns host memory; free it with shampoo_plan_destroy. */
 SHP_API shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
                                shp_plan** plan_out);
+
+/* shampoo_plan_create with flags.  SHP_PLAN_LAYERWISE stacks per layer:
+ * gradient buckets are keyed by (layer, rows, cols) and factor buckets by
+ * (layer, n), the "layerwise" stacking the DASH paper compares with its
+ * GPU-level stacking (§4 Blocking Strategy); the order inside a bucket is
+ * unchanged.  flags 0 is shampoo_plan_create; unknown bits return
+ * SHP_ERR_INVALID_ARG.  The paper has no flag: it names the two variants. */
+#define SHP_PLAN_LAYERWISE 1
+SHP_API shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int32_t n_layers,
+                                          int32_t block_size, int32_t flags, shp_plan** plan_out);
 SHP_API void shampoo_plan_destroy(shp_plan* plan);
 
 /* Table sizes: number of blocks, of gradient buckets, of factor buckets, and

@@ -23,7 +23,8 @@ BLOCK_FIELDS = 13
 
 EXPORTS = [
     "shampoo_last_error", "shampoo_version", "shampoo_launch_count", "shampoo_device_error",
-    "shampoo_plan_create", "shampoo_plan_destroy", "shampoo_plan_sizes", "shampoo_plan_tables",
+    "shampoo_plan_create", "shampoo_plan_create_ex", "shampoo_plan_destroy", "shampoo_plan_sizes",
+    "shampoo_plan_tables",
     "shampoo_plan_bind", "shampoo_stack_blocks",
     "shampoo_update_stats_workspace_bytes", "shampoo_update_stats",
     "shampoo_inv_root_workspace_bytes", "shampoo_inv_root", "shampoo_inv_root_static",
@@ -57,6 +58,7 @@ def lib() -> ctypes.CDLL:
         "shampoo_launch_count": (ctypes.c_uint64, []),
         "shampoo_device_error": (c_int32, [P(c_int32)]),
         "shampoo_plan_create": (c_int32, [P(c_int32), P(c_int32), c_int32, c_int32, P(c_void_p)]),
+        "shampoo_plan_create_ex": (c_int32, [P(c_int32), P(c_int32), c_int32, c_int32, c_int32, P(c_void_p)]),
         "shampoo_plan_destroy": (None, [c_void_p]),
         "shampoo_plan_sizes": (c_int32, [c_void_p, P(c_int32), P(c_int32), P(c_int32), P(c_size_t)]),
         "shampoo_plan_tables": (c_int32, [c_void_p, P(c_int32), P(c_int32), P(c_int32)]),
@@ -138,15 +140,16 @@ def device_error() -> int:
 
 
 class Plan:
-    """Host block plan (shampoo_plan_create) plus its bound device tables."""
+    """Host block plan (shampoo_plan_create_ex) plus its bound device tables;
+    ``layerwise`` stacks per layer (SHP_PLAN_LAYERWISE)."""
 
-    def __init__(self, shapes, block_size: int):
+    def __init__(self, shapes, block_size: int, layerwise: bool = False):
         self.shapes = [(int(m), int(n)) for (m, n) in shapes]
         rows = (c_int32 * len(self.shapes))(*[m for m, _ in self.shapes])
         cols = (c_int32 * len(self.shapes))(*[n for _, n in self.shapes])
         h = c_void_p()
-        _check(lib().shampoo_plan_create(rows, cols, len(self.shapes), int(block_size), ctypes.byref(h)),
-               "shampoo_plan_create")
+        _check(lib().shampoo_plan_create_ex(rows, cols, len(self.shapes), int(block_size), 1 if layerwise else 0,
+                                            ctypes.byref(h)), "shampoo_plan_create_ex")
         self.handle = h
         nb, ng, nf, db = c_int32(), c_int32(), c_int32(), c_size_t()
         _check(lib().shampoo_plan_sizes(h, ctypes.byref(nb), ctypes.byref(ng), ctypes.byref(nf), ctypes.byref(db)),

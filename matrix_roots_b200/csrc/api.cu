@@ -487,7 +487,14 @@ shp_status shampoo_device_error(int32_t* out) {
 
 shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
                                shp_plan** plan_out) {
+  return shampoo_plan_create_ex(rows, cols, n_layers, block_size, 0, plan_out);
+}
+
+shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
+                                  int32_t flags, shp_plan** plan_out) {
   if (!plan_out) return fail(SHP_ERR_INVALID_ARG, "plan_out is NULL");
+  if (flags & ~SHP_PLAN_LAYERWISE) return fail(SHP_ERR_INVALID_ARG, "unknown plan flags 0x%x", flags);
+  const bool layerwise = (flags & SHP_PLAN_LAYERWISE) != 0;
   *plan_out = nullptr;
   if (n_layers < 1 || !rows || !cols) return fail(SHP_ERR_INVALID_ARG, "need n_layers >= 1 and rows/cols arrays");
   if (block_size < 0) return fail(SHP_ERR_INVALID_ARG, "block_size must be >= 0");
@@ -499,14 +506,17 @@ shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t
   p->cols.assign(cols, cols + n_layers);
   p->block_size = block_size;
   std::vector<int> rs, cs;
-  std::vector<int> fkey;  // factor bucket n values in order
+  std::vector<int> fkey, flayer;  // factor bucket n values (and layers, when layerwise) in order
+  std::vector<int> glayer;        // gradient bucket layers, when layerwise
+  int cur_layer = 0;
   auto fslot = [&](int n, int32_t* bucket, int32_t* index) {
     int b = -1;
     for (size_t i = 0; i < fkey.size(); ++i)
-      if (fkey[i] == n) b = (int)i;
+      if (fkey[i] == n && (!layerwise || flayer[i] == cur_layer)) b = (int)i;
     if (b < 0) {
       b = (int)fkey.size();
       fkey.push_back(n);
+      flayer.push_back(cur_layer);
       p->fb.push_back(n);
       p->fb.push_back(0);
     }
@@ -514,6 +524,7 @@ shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t
     *index = p->fb[2 * b + 1]++;
   };
   for (int l = 0; l < n_layers; ++l) {
+    cur_layer = l;
     split_dim(rows[l], block_size, rs);
     split_dim(cols[l], block_size, cs);
     const size_t first = p->blocks.size();
@@ -528,9 +539,10 @@ shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t
         }
         int g = -1;
         for (int i = 0; i < (int)p->gb.size() / 3; ++i)
-          if (p->gb[3 * i] == r && p->gb[3 * i + 1] == c) g = i;
+          if (p->gb[3 * i] == r && p->gb[3 * i + 1] == c && (!layerwise || glayer[i] == l)) g = i;
         if (g < 0) {
           g = (int)p->gb.size() / 3;
+          glayer.push_back(l);
           p->gb.push_back(r);
           p->gb.push_back(c);
           p->gb.push_back(0);

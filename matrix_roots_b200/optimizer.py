@@ -45,6 +45,7 @@ class ShampooConfig:
     precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...; statistics every step
     root_p: int = 4             # inverse p-th roots, p in (2, 4, 8)
     graph: bool = False         # replay the launches before the graft step as a CUDA graph
+    layerwise: bool = False     # stack per layer instead of across all layers
 
 
 class BlockedShampoo:
@@ -53,7 +54,7 @@ class BlockedShampoo:
         self.cfg = cfg
         self.device = torch.device(device)
         self.shapes = [(int(m), int(n)) for m, n in shapes]
-        self.plan = B.Plan(self.shapes, cfg.block_size).bind(self.device)
+        self.plan = B.Plan(self.shapes, cfg.block_size, cfg.layerwise).bind(self.device)
         t = self.plan.tables()
         self.tables = t
         f32 = dict(dtype=torch.float32, device=self.device)

@@ -99,7 +99,7 @@ def split_dim(d: int, block_size: int) -> list[int]:
     return sizes
 
 
-def plan_blocks(shapes, block_size: int) -> dict:
+def plan_blocks(shapes, block_size: int, layerwise: bool = False) -> dict:
     """Partition every layer into blocks and assign them to stacks.
 
     Returns int32 tables:
@@ -107,7 +107,9 @@ def plan_blocks(shapes, block_size: int) -> dict:
       g_buckets (n_g, 3)  rows, cols, count of each gradient-block stack;
       f_buckets (n_f, 2)  n, count of each preconditioner-factor stack.
     Gradient blocks are bucketed by (rows, cols), factors by n ([DASH] §4);
-    the order inside buckets is reading R1.
+    the order inside buckets is reading R1.  ``layerwise`` keys the buckets
+    by layer as well ([DASH] §4: DASH-LAYERWISE stacks per layer, DASH-GPU
+    across all layers of a GPU).
     """
     blocks = []
     g_key_to_id: dict = {}
@@ -115,11 +117,12 @@ def plan_blocks(shapes, block_size: int) -> dict:
     f_key_to_id: dict = {}
     f_counts: list = []
 
-    def f_slot(n):
-        if n not in f_key_to_id:
-            f_key_to_id[n] = len(f_counts)
+    def f_slot(n, li):
+        key = (li, n) if layerwise else n
+        if key not in f_key_to_id:
+            f_key_to_id[key] = len(f_counts)
             f_counts.append([n, 0])
-        b = f_key_to_id[n]
+        b = f_key_to_id[key]
         idx = f_counts[b][1]
         f_counts[b][1] += 1
         return b, idx
@@ -132,7 +135,7 @@ def plan_blocks(shapes, block_size: int) -> dict:
         for br, r in enumerate(rs):
             col0 = 0
             for bc, c in enumerate(cs):
-                key = (r, c)
+                key = (li, r, c) if layerwise else (r, c)
                 if key not in g_key_to_id:
                     g_key_to_id[key] = len(g_counts)
                     g_counts.append([r, c, 0])
@@ -143,9 +146,9 @@ def plan_blocks(shapes, block_size: int) -> dict:
                 col0 += c
             row0 += r
         for blk in layer_blocks:          # all left factors of the layer, row-major
-            blk[9], blk[10] = f_slot(blk[5])
+            blk[9], blk[10] = f_slot(blk[5], li)
         for blk in layer_blocks:          # then all right factors, row-major
-            blk[11], blk[12] = f_slot(blk[6])
+            blk[11], blk[12] = f_slot(blk[6], li)
         blocks += layer_blocks
     return {
         "blocks": np.asarray(blocks, dtype=np.int32).reshape(-1, len(BLOCK_FIELDS)),

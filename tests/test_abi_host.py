@@ -55,11 +55,12 @@ SHAPE_CASES = [
 ]
 
 
+@pytest.mark.parametrize("layerwise", [False, True])
 @pytest.mark.parametrize("shapes,bs", SHAPE_CASES)
-def test_plan_tables_bit_exact_with_oracle(shapes, bs):
-    plan = B.Plan(shapes, bs)
+def test_plan_tables_bit_exact_with_oracle(shapes, bs, layerwise):
+    plan = B.Plan(shapes, bs, layerwise)
     got = plan.tables()
-    ref = O.plan_blocks(shapes, bs)
+    ref = O.plan_blocks(shapes, bs, layerwise)
     for k in ("blocks", "g_buckets", "f_buckets"):
         assert got[k].dtype == np.int32
         assert np.array_equal(got[k], ref[k]), k
@@ -72,10 +73,19 @@ def test_plan_random_shapes_bit_exact():
         bs = int(rng.choice([0, 64, 128, 500, 1024]))
         if bs == 0:
             shapes = [(min(m, 4096), min(n, 4096)) for m, n in shapes]
-        got = B.Plan(shapes, bs).tables()
-        ref = O.plan_blocks(shapes, bs)
+        lw = bool(rng.integers(0, 2))
+        got = B.Plan(shapes, bs, lw).tables()
+        ref = O.plan_blocks(shapes, bs, lw)
         for k in ("blocks", "g_buckets", "f_buckets"):
-            assert np.array_equal(got[k], ref[k]), (shapes, bs, k)
+            assert np.array_equal(got[k], ref[k]), (shapes, bs, lw, k)
+
+
+def test_plan_unknown_flags_refused():
+    L = B.lib()
+    rows = (ctypes.c_int32 * 1)(64)
+    cols = (ctypes.c_int32 * 1)(64)
+    h = ctypes.c_void_p()
+    assert L.shampoo_plan_create_ex(rows, cols, 1, 64, 2, ctypes.byref(h)) == B.SHP_ERR_INVALID_ARG
 
 
 def test_plan_rejects_bad_input():

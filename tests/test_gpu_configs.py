@@ -96,6 +96,36 @@ def test_cuda_graph_step_matches_direct_launches():
     assert np.array_equal(res[0], res[1])
 
 
+def test_layerwise_stacking_matches_global_stacking():
+    """Stacking blocks per layer instead of across layers ([DASH] §4,
+    Blocking Strategy) changes only which launch a block rides in: every
+    block's factors, root, direction and graft are its own, so the weights
+    after 3 steps agree (four layers with shared and ragged block shapes,
+    block size 64, AdaGrad graft).  Per-matrix sums of squares are gathered
+    with atomic adds, whose order may differ between launches, so the bound
+    is a few float32 ulps rather than bit equality."""
+    import torch
+    shapes = [(128, 256), (256, 128), (200, 136), (128, 128)]
+    rng = np.random.default_rng(11)
+    G = [[rng.standard_normal(s).astype(np.float32) for s in shapes] for _ in range(3)]
+    res = []
+    for layerwise in (False, True):
+        cfg = ShampooConfig(block_size=64, beta2=0.999, alpha=1.0, eps=1e-6, method="ndb", iters=20, dtype="fp32",
+                            scaling="frobenius", graft="adagrad", lr=0.05, layerwise=layerwise)
+        opt = BlockedShampoo(shapes, cfg)
+        n_fb = len(opt.plan.tables()["f_buckets"])
+        Wd = [torch.zeros(s, device="cuda") for s in shapes]
+        for t in range(3):
+            opt.step(Wd, [to_dev(g) for g in G[t]])
+        torch.cuda.synchronize()
+        res.append(([w.cpu().numpy() for w in Wd], n_fb))
+    assert res[1][1] > res[0][1]  # more, smaller stacks
+    for a, b in zip(res[0][0], res[1][0]):
+        assert np.isfinite(a).all() and np.abs(a).max() > 0
+        print(f"layerwise vs global: {int((a != b).sum())} of {a.size} entries differ, rel {rel(b, a):.1e}")
+        assert rel(b, a) < 1e-6
+
+
 def test_stale_roots_every_third_step():
     """Preconditioner frequency f = 3 on the tiny dense workload (6 steps,
     NDB-20 FP32): statistics every step, roots on steps 1 and 4 only.  As for

@@ -552,3 +552,28 @@ def test_ndb_root_power_chain(p):
     assert O.rel_fro(O.ndb_inv_root_replay(L, 1e-6, s, 25, p), X) < 1e-10
     # X^p (L + eps I) = I
     assert np.linalg.norm(np.linalg.matrix_power(X, p) @ (L + 1e-6 * np.eye(12)) - np.eye(12)) < 1e-9
+
+
+def test_plan_layerwise_is_per_layer_global_stacking():
+    """Layerwise stacking ([DASH] §4: DASH-LAYERWISE stacks per layer): a
+    single layer plans exactly as with stacking across layers, and for
+    several layers every bucket holds one layer's blocks, in the order and
+    with the counts that layer's own plan gives."""
+    one = [(4096, 1024)]
+    a, b = O.plan_blocks(one, 1024), O.plan_blocks(one, 1024, layerwise=True)
+    for k in ("blocks", "g_buckets", "f_buckets"):
+        assert np.array_equal(a[k], b[k])
+    shapes = [(300, 200), (200, 300), (128, 128), (300, 200)]
+    lw = O.plan_blocks(shapes, 128, layerwise=True)
+    gb_off = fb_off = 0
+    for li, shp in enumerate(shapes):
+        own = O.plan_blocks([shp], 128)
+        mine = lw["blocks"][lw["blocks"][:, 0] == li]
+        assert np.array_equal(mine[:, 1:7], own["blocks"][:, 1:7])
+        assert np.array_equal(mine[:, [7, 9, 11]] - [gb_off, fb_off, fb_off], own["blocks"][:, [7, 9, 11]])
+        assert np.array_equal(mine[:, [8, 10, 12]], own["blocks"][:, [8, 10, 12]])
+        assert np.array_equal(lw["g_buckets"][gb_off:gb_off + len(own["g_buckets"])], own["g_buckets"])
+        assert np.array_equal(lw["f_buckets"][fb_off:fb_off + len(own["f_buckets"])], own["f_buckets"])
+        gb_off += len(own["g_buckets"])
+        fb_off += len(own["f_buckets"])
+    assert gb_off == len(lw["g_buckets"]) and fb_off == len(lw["f_buckets"])

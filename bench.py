@@ -451,7 +451,7 @@ def run_ours(args, cfg):
                          "fp16": "f16", "bf16": "bf16"}[args.dtype],
                "data": "synthetic",
                "config": dict(arm_config(cfg, n_blocks, sum(int(c) for _, c in opt.tables["f_buckets"]), world),
-                              cuda_graph=bool(args.graph), stacking="layerwise" if args.layerwise else "gpu"),
+                              cuda_graph=bool(args.graph), stacking="layerwise" if args.layerwise else "global"),
                "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
                "clocks": clocks.summary()}
         if world == 1 and not args.no_cpu:

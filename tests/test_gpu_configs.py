@@ -103,14 +103,17 @@ def test_layerwise_stacking_matches_global_stacking():
     after 3 steps agree (four layers with shared and ragged block shapes,
     block size 64, AdaGrad graft).  Per-matrix sums of squares are gathered
     with atomic adds, whose order may differ between launches, so the bound
-    is a few float32 ulps rather than bit equality."""
+    is a few float32 ulps rather than bit equality.  Damping 1e-2: the 64x8
+    blocks give rank-deficient 64x64 factors, and with 1e-6 their condition
+    number (about 3e8) is past what Newton-DB survives in float32; the
+    oracle's float32 model overflows there as well."""
     import torch
     shapes = [(128, 256), (256, 128), (200, 136), (128, 128)]
     rng = np.random.default_rng(11)
     G = [[rng.standard_normal(s).astype(np.float32) for s in shapes] for _ in range(3)]
     res = []
     for layerwise in (False, True):
-        cfg = ShampooConfig(block_size=64, beta2=0.999, alpha=1.0, eps=1e-6, method="ndb", iters=20, dtype="fp32",
+        cfg = ShampooConfig(block_size=64, beta2=0.999, alpha=1.0, eps=1e-2, method="ndb", iters=20, dtype="fp32",
                             scaling="frobenius", graft="adagrad", lr=0.05, layerwise=layerwise)
         opt = BlockedShampoo(shapes, cfg)
         n_fb = len(opt.plan.tables()["f_buckets"])

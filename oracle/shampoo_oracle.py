@@ -49,6 +49,13 @@ R12 Root power p: p in {2, 4, 8} ([Notes] "Spreading the preconditioners":
 R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
     Hyperparameters: preconditioning_compute_steps; [DASH] §1).
+R13 Layerwise stacking: the R1 partition and order with buckets keyed by
+    (layer, shape), so no stack mixes layers ([DASH] §4, Stacking strategy).
+R14 Warm-started coupled Newton ([Notes] "Roots on idle CPUs": the roots
+    start from the previous root): X_0 = the previous root, M_0 = X_0^p A
+    (the iteration's invariant M = X^p A), no scaling, then the R5 update.
+    Exact when X_0 commutes with A; otherwise the result is the same
+    iteration's, not A^{-1/p}.
 
 Parity unpinned: the power-iteration iteration count (R7: no page fixes it),
 the step-count example of [DASH] §3 (Frobenius scaling 5 -> 15 steps).
@@ -64,7 +71,7 @@ __all__ = [
     "update_stats", "spd_power", "inv_root_exact",
     "frobenius_scale", "power_iteration_scale",
     "ndb_matrix", "ndb_calls", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
-    "cn_matrix", "cn_inv_root", "cn_scalar", "cn_inv_root_replay",
+    "cn_matrix", "cn_inv_root", "cn_inv_root_warm", "cn_scalar", "cn_inv_root_replay",
     "cheb_coefficients", "clenshaw_scalar", "cheb_matrix", "cheb_inv_root", "cheb_inv_root_replay",
     "inv_root", "precondition", "graft_update", "ShampooState", "compute_roots", "shampoo_step",
     "rel_fro", "round_mantissa", "truncate_mantissa", "precision_floor",
@@ -380,14 +387,14 @@ def ndb_inv_root_replay(L, eps: float, s: float, iters: int, p: int = 4):
 #     Higham / Iannazzo; [DASH] §1, §5)
 # --------------------------------------------------------------------------
 
-def cn_matrix(M0, iters: int, p: int = 4, prec=None):
-    """Coupled Newton for M0^{-1/p}: X0 = I, T = ((p+1)I - M)/p, X <- X T,
-    M <- T^p M.  Returns (X, matmuls); T^p by binary powering (2 products
-    for p = 4, so 4 matmuls per iteration)."""
+def cn_matrix(M0, iters: int, p: int = 4, prec=None, X0=None):
+    """Coupled Newton for M0^{-1/p}: X0 = I (or the given start), T =
+    ((p+1)I - M)/p, X <- X T, M <- T^p M.  Returns (X, matmuls); T^p by
+    binary powering (2 products for p = 4, so 4 matmuls per iteration)."""
     mul, st = _model(prec)
     M = st(np.asarray(M0, dtype=np.float64))
     I = st(np.eye(M.shape[0]))
-    X = I.copy()
+    X = I.copy() if X0 is None else st(np.asarray(X0, dtype=np.float64))
     mm = 0
     for _ in range(iters):
         T = st(((p + 1) * I - M) / p)
@@ -416,6 +423,17 @@ def cn_inv_root(L, eps: float, s: float, iters: int, p: int = 4, prec=None):
     A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
     X, mm = cn_matrix(st(A / s), iters, p, prec)
     return s ** (-1.0 / p) * np.asarray(X, np.float64), mm
+
+
+def cn_inv_root_warm(L, X0, eps: float, iters: int, p: int = 4):
+    """(L + eps I)^{-1/p} by coupled Newton warm-started from a previous root
+    X0 (reading R14): M_0 = X0^p (L + eps I), X_0 = X0, then the update of
+    ``cn_matrix``; no scaling and no final multiplier.  Float64."""
+    A = np.asarray(L, dtype=np.float64) + eps * np.eye(L.shape[0])
+    X0 = np.asarray(X0, dtype=np.float64)
+    M0 = np.linalg.matrix_power(X0, p) @ A
+    X, _ = cn_matrix(M0, iters, p, X0=X0)
+    return np.asarray(X, np.float64)
 
 
 def cn_scalar(a, iters: int, p: int = 4):

@@ -577,3 +577,73 @@ def test_plan_layerwise_is_per_layer_global_stacking():
         gb_off += len(own["g_buckets"])
         fb_off += len(own["f_buckets"])
     assert gb_off == len(lw["g_buckets"]) and fb_off == len(lw["f_buckets"])
+
+
+# ---- warm-started coupled Newton (reading R14) ------------------------------
+
+def _haar(n, rng):
+    q, r = np.linalg.qr(rng.standard_normal((n, n)))
+    return q * np.sign(np.diag(r))
+
+
+@pytest.mark.parametrize("p", [2, 4, 8])
+def test_cn_warm_from_exact_root_is_a_fixed_point(p):
+    """Started at the exact root, M_0 = I, so T = I and every iterate stays
+    at the start: the exact (L + eps I)^{-1/p} is a fixed point."""
+    rng = np.random.default_rng(5)
+    Q = _haar(24, rng)
+    lam = 10.0 ** rng.uniform(-3, 1, 24)
+    L = (Q * lam) @ Q.T
+    X0 = (Q * (lam + 1e-4) ** (-1.0 / p)) @ Q.T
+    X = O.cn_inv_root_warm(L, X0, 1e-4, 6, p)
+    assert O.rel_fro(X, X0) < 1e-12
+
+
+@pytest.mark.parametrize("p", [2, 4, 8])
+def test_cn_warm_commuting_start_is_the_scalar_recurrence(p):
+    """A start that shares L's eigenvectors keeps the iteration diagonal in
+    that basis: eigenvalue by eigenvalue x = x0 * (cold scalar recurrence on
+    m0 = x0^p a).  Checks the matrix products (order, powers, the M_0
+    product) against the scalar update."""
+    rng = np.random.default_rng(6)
+    Q = _haar(20, rng)
+    lam = 10.0 ** rng.uniform(-2, 0, 20)
+    L = (Q * lam) @ Q.T
+    x0 = (lam * rng.uniform(0.7, 1.4, 20)) ** (-1.0 / p)
+    X0 = (Q * x0) @ Q.T
+    a = lam + 1e-3
+    x = x0 * O.cn_scalar(x0 ** p * a, 5, p)
+    assert O.rel_fro(O.cn_inv_root_warm(L, X0, 1e-3, 5, p), (Q * x) @ Q.T) < 1e-12
+
+
+def test_cn_warm_from_scaled_identity_is_cold_cn():
+    """X0 = s^{-1/p} I commutes with everything: M_0 = A/s and X_k =
+    s^{-1/p} times the cold iterate, i.e. the cold coupled Newton with
+    scale s."""
+    rng = np.random.default_rng(7)
+    B = rng.standard_normal((32, 48))
+    L = B @ B.T
+    s = O.frobenius_scale(L, 1e-6)
+    X0 = s ** (-0.25) * np.eye(32)
+    cold, _ = O.cn_inv_root(L, 1e-6, s, 9)
+    assert O.rel_fro(O.cn_inv_root_warm(L, X0, 1e-6, 9), cold) < 1e-12
+
+
+def test_cn_warm_start_improves_a_stale_root():
+    """One statistics update later (beta2 = 0.999, one new gradient), the
+    previous exact root does not commute with the new factor, so the warm
+    iteration settles at its own fixed point instead of the exact root: it
+    gets there within three iterations and is better than the stale root
+    it started from."""
+    rng = np.random.default_rng(8)
+    G = [rng.standard_normal((64, 256)) for _ in range(2)]
+    L0 = G[0] @ G[0].T
+    L1 = 0.999 * L0 + G[1] @ G[1].T * 1e-3
+    eps = 1e-3
+    exact = O.inv_root_exact(L1, eps)
+    X0 = O.inv_root_exact(L0, eps)
+    e_start = O.rel_fro(X0, exact)
+    e3 = O.rel_fro(O.cn_inv_root_warm(L1, X0, eps, 3), exact)
+    e10 = O.rel_fro(O.cn_inv_root_warm(L1, X0, eps, 10), exact)
+    assert e3 < 0.5 * e_start
+    assert abs(e3 - e10) < 1e-3 * e10

@@ -236,6 +236,35 @@ SHP_API shp_status shampoo_inv_root_static(const float* A, int32_t count, int32_
                                            int32_t pi_vectors, int32_t pi_iters, const float* pi_starts,
                                            float* X_out, float* scale_out, int32_t* status_out, void* stream);
 
+/* Coupled Newton warm-started from a previous root   ([Notes] "Roots on
+ * idle CPUs": coupled Newton, started from the previous root)
+ *   A = L + eps I; X0 = X0_in; M0 = X0^p A (X0^p by squarings);
+ *   T = ((p+1)I - M)/p, X <- X T, M <- T^p M for iters iterations; no
+ *   scaling and no final multiplier.  When X0 commutes with L (shares its
+ *   eigenvectors) the iterates converge to A^(-1/p); a root of an earlier L
+ *   does not commute with the new one, and the iteration then settles at
+ *   X0 (X0^p A)^(-1/p), a fixed point of its own, within a few iterations.
+ *   It converges when the eigenvalues of M0 lie in (0, p + 1).  Chaining
+ *   it step after step from its own results compounds that error (it
+ *   diverged within 4 to 6 chained refreshes of a growing Gram factor,
+ *   in float64 as well), so a cold root has to be taken now and then. 
+ * A, X0: device (count, n, n) float32, row-major, 16-byte aligned; X0 is
+ *   read once at the start, so X_out may be X0 (in-place refresh).
+ * X_out: device (count, n, n) float32; status_out [count] as for
+ *   shampoo_inv_root.  p in {2, 4, 8}; dtype as for shampoo_inv_root;
+ *   1 <= iters <= 1000; sizes as for shampoo_inv_root.
+ * Products: 4 iters for p = 4 (3 iters + 1 for p = 2, 5 iters + 3 for
+ *   p = 8), each a (count, n, n) GEMM.
+ * Errors (nothing enqueued): SHP_ERR_INVALID_ARG for NULL pointers, bad
+ *   dtype, eps < 0 or not finite, misaligned pointers; SHP_ERR_SHAPE for
+ *   n or count out of range; SHP_ERR_UNSUPPORTED for other p;
+ *   SHP_ERR_WORKSPACE when ws_bytes is below
+ *   shampoo_inv_root_warm_workspace_bytes (0 for invalid sizes). */
+SHP_API size_t shampoo_inv_root_warm_workspace_bytes(int32_t count, int32_t n, int32_t dtype);
+SHP_API shp_status shampoo_inv_root_warm(const float* A, const float* X0, int32_t count, int32_t n, float eps,
+                                         int32_t p, int32_t iters, int32_t dtype, float* X_out,
+                                         int32_t* status_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------
  * a7  Two-sided preconditioning   ([DASH] §2)
  *   D_b = X_L(b) G_b X_R(b)   for every gradient block b

@@ -28,6 +28,7 @@ EXPORTS = [
     "shampoo_plan_bind", "shampoo_stack_blocks",
     "shampoo_update_stats_workspace_bytes", "shampoo_update_stats",
     "shampoo_inv_root_workspace_bytes", "shampoo_inv_root", "shampoo_inv_root_static",
+    "shampoo_inv_root_warm_workspace_bytes", "shampoo_inv_root_warm",
     "shampoo_precondition_workspace_bytes", "shampoo_precondition",
     "shampoo_graft_step_workspace_bytes", "shampoo_graft_step",
 ]
@@ -74,6 +75,9 @@ def lib() -> ctypes.CDLL:
         "shampoo_inv_root_static": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_int32, c_int32, c_int32,
                                               c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p,
                                               c_void_p, c_void_p]),
+        "shampoo_inv_root_warm_workspace_bytes": (c_size_t, [c_int32] * 3),
+        "shampoo_inv_root_warm": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_float, c_int32, c_int32,
+                                            c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
         "shampoo_precondition_workspace_bytes": (c_size_t, [c_void_p, c_int32]),
         "shampoo_precondition": (c_int32, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), c_void_p, c_int32,
                                            c_void_p, c_size_t, c_void_p]),
@@ -223,6 +227,26 @@ def inv_root(A, eps: float, method="ndb", iters: int = 20, dtype="fp32", scaling
                                   _ptr(pi_starts), _ptr(X), _ptr(s), _ptr(st), _ptr(workspace), workspace.numel(),
                                   _stream(stream)), "shampoo_inv_root")
     return X, s, st
+
+
+def inv_root_warm_workspace_bytes(count: int, n: int, dtype="fp32") -> int:
+    return int(lib().shampoo_inv_root_warm_workspace_bytes(count, n, _enum(DTYPES, dtype)))
+
+
+def inv_root_warm(A, X0, eps: float, iters: int = 3, dtype="fp32", p: int = 4, out=None, status_out=None,
+                  workspace=None, stream=None):
+    """Coupled Newton warm-started from the previous roots X0 (same shape as
+    A); returns (X, status).  ``out`` may be X0."""
+    import torch
+    count, n = int(A.shape[0]), int(A.shape[1])
+    X = out if out is not None else torch.empty_like(A)
+    st = status_out if status_out is not None else torch.empty(count, dtype=torch.int32, device=A.device)
+    if workspace is None:
+        workspace = _workspace(inv_root_warm_workspace_bytes(count, n, dtype), A.device)
+    _check(lib().shampoo_inv_root_warm(_ptr(A), _ptr(X0), count, n, float(eps), int(p), int(iters),
+                                       _enum(DTYPES, dtype), _ptr(X), _ptr(st), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "shampoo_inv_root_warm")
+    return X, st
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

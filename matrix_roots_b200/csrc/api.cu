@@ -384,6 +384,83 @@ shp_status run_cn(const float* A, int count, int n, float eps, int iters, int p,
   return SHP_OK;
 }
 
+// Coupled Newton warm-started from a previous root X0 (the iteration the
+// "Shampoo" notes describe under "Roots on idle CPUs"): X_0 = X0 and
+// M_0 = X0^p (L + eps I), the invariant M = X^p A of the cold start, with no
+// scaling and no final multiplier.  Then the update of run_cn, where the
+// first X product is a real GEMM.  Products: X0^2 (X0^4, X0^8 by squaring),
+// X0^p A, then X T, T T, (T^2 T^2, T^4 T^4), T^p M per iteration and X T
+// alone in the last one: 4 k for p = 4.
+shp_status run_cn_warm(const float* A, const float* X0, int count, int n, float eps, int iters, int p, Prec pr,
+                       RootBufs& r, float* X, int* status, cudaStream_t st) {
+  Planes* Xp = r.Y;
+  Planes* Mp = r.Z;
+  const long long bs = (long long)n * n;
+  const float ip = 1.f / (float)p, pp = (float)(p + 1) / (float)p;
+  GEMM_TRY(launch_to_planes(X0, n, bs, nullptr, count, n, n, 1.f, 0.f, 0.f, nullptr, Xp[0], pr, st));
+  GEMM_TRY(launch_to_planes(A, n, bs, nullptr, count, n, n, 1.f, eps, 0.f, nullptr, Mp[1], pr, st));
+  GemmGroup g = group(n, n, n, &Xp[0], 0, &Xp[0], 1);  // X0^2
+  g.epi.O = as_out(r.T2, false);
+  GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
+  Planes* Xpow = &r.T2;
+  if (p >= 4) {
+    g = group(n, n, n, &r.T2, 0, &r.T2, 1);  // X0^4
+    g.epi.O = as_out(r.T4, false);
+    GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
+    Xpow = &r.T4;
+  }
+  if (p == 8) {
+    g = group(n, n, n, &r.T4, 0, &r.T4, 1);  // X0^8
+    g.epi.O = as_out(r.T2, false);
+    GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
+    Xpow = &r.T2;
+  }
+  g = group(n, n, n, Xpow, 0, &Mp[1], 1);  // M_0 = X0^p A, T_0 = ((p+1) I - M_0)/p
+  g.epi.O = as_out(Mp[0], false);
+  g.epi.X = as_out(r.T, false);
+  g.epi.alpha2 = -ip;
+  g.epi.gamma2 = pp;
+  GEMM_TRY(launch_gemm(&g, 1, count, pr, st));
+  int cx = 0, cm = 0;
+  for (int it = 1; it <= iters; ++it) {
+    GemmGroup gs[2];
+    gs[0] = group(n, n, n, &Xp[cx], 0, &r.T, 1);  // X' = X T
+    if (it == iters) {
+      gs[0].epi.O = final_out(X, n);
+      gs[0].epi.root_p = p;
+      gs[0].epi.status = status;
+      GEMM_TRY(launch_gemm(gs, 1, count, pr, st));
+      break;
+    }
+    gs[0].epi.O = as_out(Xp[1 - cx], false);
+    gs[1] = group(n, n, n, &r.T, 0, &r.T, 1);  // T^2
+    gs[1].epi.O = as_out(r.T2, false);
+    GEMM_TRY(launch_gemm(gs, 2, count, pr, st));
+    cx = 1 - cx;
+    Planes* Tp = &r.T2;
+    if (p >= 4) {
+      GemmGroup g4 = group(n, n, n, &r.T2, 0, &r.T2, 1);
+      g4.epi.O = as_out(r.T4, false);
+      GEMM_TRY(launch_gemm(&g4, 1, count, pr, st));
+      Tp = &r.T4;
+    }
+    if (p == 8) {
+      GemmGroup g8 = group(n, n, n, &r.T4, 0, &r.T4, 1);
+      g8.epi.O = as_out(r.T2, false);
+      GEMM_TRY(launch_gemm(&g8, 1, count, pr, st));
+      Tp = &r.T2;
+    }
+    GemmGroup gm = group(n, n, n, Tp, 0, &Mp[cm], 1);  // M' = T^p M, next T
+    gm.epi.O = as_out(Mp[1 - cm], false);
+    gm.epi.X = as_out(r.T, false);
+    gm.epi.alpha2 = -ip;
+    gm.epi.gamma2 = pp;
+    GEMM_TRY(launch_gemm(&gm, 1, count, pr, st));
+    cm = 1 - cm;
+  }
+  return SHP_OK;
+}
+
 // Chebyshev approximation with the optimised matrix Clenshaw recurrence
 // ("DASH", A.2): d - 1 matmuls for degree d.
 shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int p, Prec pr, RootBufs& r,
@@ -795,6 +872,32 @@ shp_status shampoo_inv_root(const float* A, int32_t count, int32_t n, float eps,
   if (method == SHP_METHOD_NDB) return run_ndb(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
   if (method == SHP_METHOD_CN) return run_cn(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
   return run_cheb(A, count, n, eps, iters, p, pr, r, scale_out, X_out, status_out, st);
+}
+
+size_t shampoo_inv_root_warm_workspace_bytes(int32_t count, int32_t n, int32_t dtype) {
+  if (check_root_args(count, n, 4, SHP_METHOD_CN, 1, dtype, SHP_SCALE_FROBENIUS, 16)) return 0;
+  Carver c(nullptr);
+  carve_roots(c, count, n, SHP_METHOD_CN, (Prec)dtype, SHP_SCALE_FROBENIUS, 16);
+  return c.off;
+}
+
+shp_status shampoo_inv_root_warm(const float* A, const float* X0, int32_t count, int32_t n, float eps, int32_t p,
+                                 int32_t iters, int32_t dtype, float* X_out, int32_t* status_out, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  shp_status s = check_root_args(count, n, p, SHP_METHOD_CN, iters, dtype, SHP_SCALE_FROBENIUS, 16);
+  if (s) return s;
+  if (!A || !X0 || !X_out || !status_out || !workspace)
+    return fail(SHP_ERR_INVALID_ARG, "A, X0, X_out, status_out and workspace must be non-NULL");
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SHP_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(A) & 15) ||
+      (reinterpret_cast<uintptr_t>(X0) & 15) || (reinterpret_cast<uintptr_t>(X_out) & 15))
+    return fail(SHP_ERR_INVALID_ARG, "workspace must be 256-byte aligned, A, X0 and X_out 16-byte aligned");
+  Carver c(workspace);
+  RootBufs r = carve_roots(c, count, n, SHP_METHOD_CN, (Prec)dtype, SHP_SCALE_FROBENIUS, 16);
+  if (c.off > ws_bytes) return fail(SHP_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, c.off);
+  cudaStream_t st = as_stream(stream);
+  CUDA_TRY(launch_zero_i32(status_out, count, st));
+  return run_cn_warm(A, X0, count, n, eps, iters, p, (Prec)dtype, r, X_out, status_out, st);
 }
 
 // ---- precondition ----------------------------------------------------------

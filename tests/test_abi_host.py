@@ -164,3 +164,34 @@ def test_calls_need_a_bound_plan():
     assert L.shampoo_precondition(plan.handle, arr, arr, arr, 0x1000, 0, None, 0, None) == B.SHP_ERR_INVALID_ARG
     assert L.shampoo_graft_step(plan.handle, arr, arr, arr, 0x1000, None, None, 1, 0.1, 0.9, 0.999, 1e-8, 0.0, 1,
                                 0, None, 0, None) == B.SHP_ERR_INVALID_ARG
+
+
+def _call_warm(**over):
+    L = B.lib()
+    args = dict(A=0x1000, X0=0x2000, count=4, n=64, eps=1e-6, p=4, iters=3, dtype=0, X=0x3000, status=0x4000,
+                ws=0x10000, ws_bytes=1 << 30, stream=0)
+    args.update(over)
+    return L.shampoo_inv_root_warm(args["A"], args["X0"], args["count"], args["n"], args["eps"], args["p"],
+                                   args["iters"], args["dtype"], args["X"], args["status"], args["ws"],
+                                   args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(A=0), B.SHP_ERR_INVALID_ARG),
+    (dict(X0=0), B.SHP_ERR_INVALID_ARG),
+    (dict(X0=0x2004), B.SHP_ERR_INVALID_ARG),
+    (dict(dtype=9), B.SHP_ERR_INVALID_ARG),
+    (dict(n=6), B.SHP_ERR_SHAPE),
+    (dict(count=0), B.SHP_ERR_SHAPE),
+    (dict(p=3), B.SHP_ERR_UNSUPPORTED),
+    (dict(iters=0), B.SHP_ERR_INVALID_ARG),
+    (dict(eps=-1.0), B.SHP_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), B.SHP_ERR_WORKSPACE),
+])
+def test_inv_root_warm_rejects_before_enqueue(over, code):
+    assert _call_warm(**over) == code
+
+
+def test_inv_root_warm_workspace_is_the_cn_workspace():
+    assert B.inv_root_warm_workspace_bytes(8, 64) == B.inv_root_workspace_bytes(8, 64, "cn", "fp32")
+    assert B.inv_root_warm_workspace_bytes(8, 6) == 0

@@ -129,6 +129,42 @@ def test_layerwise_stacking_matches_global_stacking():
         assert rel(b, a) < 1e-6
 
 
+def _warm_case(n, count, seed):
+    """Factors one statistics update apart: L0 = G0 G0^T, L1 = 0.999 L0 +
+    1e-3 G1 G1^T with n x 3n Gaussian gradients, and X0 the exact root of L0
+    rounded to float32."""
+    rng = np.random.default_rng(seed)
+    L1, X0 = [], []
+    for _ in range(count):
+        G0, G1 = rng.standard_normal((n, 3 * n)), rng.standard_normal((n, 3 * n))
+        L0 = G0 @ G0.T
+        L1.append(0.999 * L0 + 1e-3 * (G1 @ G1.T))
+        X0.append(O.inv_root_exact(L0, 1e-3))
+    return np.stack(L1).astype(np.float32), np.stack(X0).astype(np.float32)
+
+
+@pytest.mark.parametrize("p", [2, 4, 8])
+@pytest.mark.parametrize("n", [128, 72])
+def test_inv_root_warm_matches_oracle(n, p):
+    """Warm-started coupled Newton (3 iterations from the previous exact
+    root) against the float64 oracle of the same iteration on the same
+    float32 inputs: stated 1e-3 (well-conditioned, kappa ~ 15).  In place
+    (X_out = X0) gives the same bits."""
+    import torch
+    L1, X0 = _warm_case(n, 5, 40 + n + p)
+    Ld, X0d = to_dev(L1), to_dev(X0)
+    X, st = B.inv_root_warm(Ld, X0d, 1e-3, 3, "fp32", p)
+    X2 = X0d.clone()
+    B.inv_root_warm(Ld, X2, 1e-3, 3, "fp32", p, out=X2)
+    torch.cuda.synchronize()
+    assert (st.cpu().numpy() == 0).all()
+    assert torch.equal(X, X2)
+    X = X.cpu().numpy()
+    for b in range(L1.shape[0]):
+        ref = O.cn_inv_root_warm(L1[b].astype(np.float64), X0[b].astype(np.float64), 1e-3, 3, p)
+        assert rel(X[b], ref) < 1e-3, (b, rel(X[b], ref))
+
+
 def test_stale_roots_every_third_step():
     """Preconditioner frequency f = 3 on the tiny dense workload (6 steps,
     NDB-20 FP32): statistics every step, roots on steps 1 and 4 only.  As for

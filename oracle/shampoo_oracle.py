@@ -49,6 +49,13 @@ R12 Root power p: p in {2, 4, 8} ([Notes] "Spreading the preconditioners":
 R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
     Hyperparameters: preconditioning_compute_steps; [DASH] §1).
+R15 EVD roots with the dampening heuristics of [DASH] B.1-B.2: the
+    eigendecomposition is taken of L + eps I, mu = its eigenvalues, and
+    lambda = mu - eps (the corrected spectrum).  corrected: (max(lambda, 0)
+    + eps)^{-1/p} (= R3); shifted-ReLU: r = max(lambda - eps, 0), r^{-1/p}
+    where r > 0 and 0 elsewhere (a rank-r_eps inverse); ABS-add:
+    (|lambda| + eps)^{-1/p}; SHMP (the Distributed Shampoo adjustment B.1
+    describes, eps added twice): mu - min(min(mu), 0) + eps.
 R13 Layerwise stacking: the R1 partition and order with buckets keyed by
     (layer, shape), so no stack mixes layers ([DASH] §4, Stacking strategy).
 R14 Warm-started coupled Newton ([Notes] "Roots on idle CPUs": the roots
@@ -68,7 +75,7 @@ import numpy as np
 
 __all__ = [
     "BLOCK_FIELDS", "split_dim", "plan_blocks", "stack_gradients", "unstack_directions",
-    "update_stats", "spd_power", "inv_root_exact",
+    "update_stats", "spd_power", "inv_root_exact", "EVD_HEURISTICS", "evd_root_factors", "evd_inv_root",
     "frobenius_scale", "power_iteration_scale",
     "ndb_matrix", "ndb_calls", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
     "cn_matrix", "cn_inv_root", "cn_inv_root_warm", "cn_scalar", "cn_inv_root_replay",
@@ -212,6 +219,38 @@ def spd_power(A, r: float, shift: float = 0.0):
 def inv_root_exact(L, eps: float, p: int = 4):
     """(L + eps I)^{-1/p} with L's eigenvalues clamped at zero (reading R3)."""
     return spd_power(L, -1.0 / p, shift=eps)
+
+
+EVD_HEURISTICS = ("corrected", "shifted_relu", "abs_add", "shmp")
+
+
+def evd_root_factors(mu, eps: float, heuristic: str, p: int = 4):
+    """f(mu) of reading R15 for the eigenvalues mu of L + eps I."""
+    mu = np.asarray(mu, dtype=np.float64)
+    lam = mu - eps
+    if heuristic == "corrected":
+        d = np.maximum(lam, 0.0) + eps
+    elif heuristic == "abs_add":
+        d = np.abs(lam) + eps
+    elif heuristic == "shmp":
+        d = mu - min(float(mu.min()), 0.0) + eps
+    elif heuristic == "shifted_relu":
+        r = np.maximum(lam - eps, 0.0)
+        out = np.zeros_like(r)
+        pos = r > 0
+        out[pos] = r[pos] ** (-1.0 / p)
+        return out
+    else:
+        raise ValueError(heuristic)
+    return d ** (-1.0 / p)
+
+
+def evd_inv_root(L, eps: float, heuristic: str = "corrected", p: int = 4):
+    """Q diag(f(mu)) Q^T from eigh(L + eps I) ([DASH] B.1-B.2, reading R15)."""
+    L = np.asarray(L, dtype=np.float64)
+    A = 0.5 * (L + L.T) + eps * np.eye(L.shape[0])
+    mu, Q = np.linalg.eigh(A)
+    return (Q * evd_root_factors(mu, eps, heuristic, p)) @ Q.T
 
 
 # --------------------------------------------------------------------------

@@ -647,3 +647,57 @@ def test_cn_warm_start_improves_a_stale_root():
     e10 = O.rel_fro(O.cn_inv_root_warm(L1, X0, eps, 10), exact)
     assert e3 < 0.5 * e_start
     assert abs(e3 - e10) < 1e-3 * e10
+
+
+# ---- EVD roots with the dampening heuristics (reading R15) -------------------
+
+def _known_spectrum(lam, seed):
+    rng = np.random.default_rng(seed)
+    q, r = np.linalg.qr(rng.standard_normal((len(lam), len(lam))))
+    Q = q * np.sign(np.diag(r))
+    return Q, (Q * np.asarray(lam, np.float64)) @ Q.T
+
+
+# L's eigenvalues, eps = 1e-2, and the diagonal each heuristic gives in
+# L's eigenbasis, written out by hand from [DASH] B.1-B.2:
+#   corrected     (max(l, 0) + eps)^(-1/4)
+#   shifted_relu  (l - eps)^(-1/4) where l > eps, else 0
+#   abs_add       (|l| + eps)^(-1/4)
+#   shmp          mu = l + eps has min 0.006 > 0, so l + 2 eps
+_LAM = [3.0, 0.5, 2e-2, 5e-3, 0.0, -4e-3]
+_EXPECT = {
+    "corrected": [3.01, 0.51, 0.03, 0.015, 0.01, 0.01],
+    "shifted_relu": [2.99, 0.49, 0.01, None, None, None],
+    "abs_add": [3.01, 0.51, 0.03, 0.015, 0.01, 0.014],
+    "shmp": [3.02, 0.52, 0.04, 0.025, 0.02, 0.016],
+}
+
+
+@pytest.mark.parametrize("heuristic", ["corrected", "shifted_relu", "abs_add", "shmp"])
+def test_evd_heuristics_on_a_known_spectrum(heuristic):
+    Q, L = _known_spectrum(_LAM, 21)
+    f = np.array([0.0 if d is None else d ** -0.25 for d in _EXPECT[heuristic]])
+    assert O.rel_fro(O.evd_inv_root(L, 1e-2, heuristic), (Q * f) @ Q.T) < 1e-10
+
+
+def test_evd_shmp_with_a_negative_damped_eigenvalue():
+    """mu_min = -0.05 + 0.01 < 0: SHMP shifts every mu by -mu_min + eps, so
+    the smallest lands on eps and the others on l + eps - mu_min + eps."""
+    lam = [2.0, 0.1, -0.05]
+    Q, L = _known_spectrum(lam, 22)
+    d = np.array([2.0 + 0.01 + 0.04 + 0.01, 0.1 + 0.01 + 0.04 + 0.01, 0.01])
+    assert O.rel_fro(O.evd_inv_root(L, 1e-2, "shmp", p=2), (Q * d ** -0.5) @ Q.T) < 1e-10
+
+
+def test_evd_corrected_is_the_exact_root_and_shifted_relu_kills_the_null_space():
+    rng = np.random.default_rng(23)
+    G = rng.standard_normal((16, 5))
+    L = G @ G.T  # rank 5 of 16
+    assert O.rel_fro(O.evd_inv_root(L, 1e-3), O.inv_root_exact(L, 1e-3)) < 1e-9
+    X = O.evd_inv_root(L, 1e-3, "shifted_relu")
+    null = np.linalg.svd(G.T)[2][5:]  # orthonormal rows spanning L's null space
+    assert np.abs(X @ null.T).max() < 1e-9 * np.abs(X).max()
+    # on the range it is (lambda - eps)^(-1/4)
+    w, U = np.linalg.eigh(L)
+    U5, w5 = U[:, -5:], w[-5:]
+    assert O.rel_fro(U5.T @ X @ U5, np.diag((w5 - 1e-3) ** -0.25)) < 1e-9

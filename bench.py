@@ -530,6 +530,88 @@ def run_spd_methods(A, count, n, args, peaks, rows):
         del ws
 
 
+EVD_HEURISTIC_NAMES = ["corrected", "shifted_relu", "abs_add", "shmp"]
+
+
+def evd_fp64_flops(n, sweeps) -> float:
+    """Float64 work of the Jacobi solves: per sweep n(n-1)/2 rotations, each
+    updating two rows and two columns of A (n element pairs each, 2 fused
+    multiply-adds per element: 8 flops per pair)."""
+    return float(np.sum(sweeps)) * (n * (n - 1) / 2) * 16.0 * n
+
+
+def run_evd(args):
+    """EVD roots against the iterative ones on C2's factor shape: 512 SPD
+    128^2 matrices Q diag(lam) Q^T, lam log-uniform in [1e-6, 1], eps = 1e-8.
+    Times shampoo_inv_root_evd for each dampening heuristic and, on the same
+    stack, Newton-DB-20 and coupled Newton-20 in FP32 (CUDA events, inputs
+    resident).  value = EVD (corrected spectrum) matrices/s; the roofline is
+    the float64 ALU work of the sweeps the solver reports, against the
+    float64 FMA rate of 148 SMs x 64 lanes at the sampled SM clock."""
+    import torch
+    from matrix_roots_b200 import binding as B
+    from matrix_roots_b200 import build
+    from matrix_roots_b200 import workloads as W
+    build.build()
+    A32, _, _ = W.spd_stack(512, 128, seed=0)
+    A = torch.from_numpy(A32).cuda()
+    count, n = A.shape[0], A.shape[1]
+    peaks = load_peaks()
+    rows = {}
+    X = torch.empty_like(A)
+    st = torch.empty(count, dtype=torch.int32, device="cuda")
+    l0 = B.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for h in EVD_HEURISTIC_NAMES:
+            for _ in range(args.warmup):
+                B.inv_root_evd(A, 1e-8, h, out=X, status_out=st)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                B.inv_root_evd(A, 1e-8, h, out=X, status_out=st)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            s_np = st.cpu().numpy()
+            sweeps = s_np >> 8
+            rows[f"evd_{h}"] = {"ms": ms, "matrices_per_s": count / (ms / 1000.0),
+                                "sweeps_mean": float(sweeps.mean()), "sweeps_max": int(sweeps.max()),
+                                "unconverged": int(((s_np & 0xff) != 0).sum()),
+                                "fp64_tflops": evd_fp64_flops(n, sweeps) / (ms / 1000.0) / 1e12}
+        for method in ("ndb", "cn"):
+            ws = torch.empty(B.inv_root_workspace_bytes(count, n, method, "fp32", "frobenius"), dtype=torch.uint8,
+                             device="cuda")
+            for _ in range(args.warmup):
+                B.inv_root(A, 1e-8, method, 20, "fp32", "frobenius", workspace=ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                B.inv_root(A, 1e-8, method, 20, "fp32", "frobenius", workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            rows[f"{method}20_fp32"] = {"ms": ms, "matrices_per_s": count / (ms / 1000.0)}
+    launches = B.launch_count() - l0
+    cs = clocks.summary()
+    ref = rows["evd_corrected"]
+    mhz = cs.get("sm_mhz") or 1965.0
+    peak = 148 * 64 * 2 * mhz * 1e6 / 1e12
+    out = {"metric": "inverse-root throughput, EVD (SPD stack)", "value": ref["matrices_per_s"],
+           "unit": "matrices/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ref["ms"],
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64 Jacobi rotations, f32 eigenvectors and roots", "data": "synthetic",
+           "config": {"workload": "spd_512x128_logunif_1e-6_1", "eps": 1e-8,
+                      "l2": "inputs 32 MB, resident in L2 (one CTA per matrix reads it once)"},
+           "roofline": {"bound": "alu", "achieved": ref["fp64_tflops"], "peak": peak, "unit": "TFLOP/s (fp64)",
+                        "frac": ref["fp64_tflops"] / peak, "traffic": None,
+                        "kernel": "evd_root_kernel (corrected spectrum)",
+                        "peak_note": "148 SMs x 64 fp64 FMA lanes x 2 x sampled SM clock"},
+           "methods": rows, "gpu_launches": launches, "clocks": cs}
+    print(json.dumps(out), flush=True)
+
+
 def run_root_stack(args):
     """Small fixed case of the dominant kernel for profilers: Newton-DB-20
     on `args.root_stack` factors L = G G^T of transformer gradient blocks
@@ -562,7 +644,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="transformer", choices=sorted(CONFIGS) + ["spd_stack"])
+    ap.add_argument("--config", default="transformer", choices=sorted(CONFIGS) + ["spd_stack", "evd_stack"])
     ap.add_argument("--dtype", default="fp32", choices=["fp32", "tf32", "fp16", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -583,6 +665,13 @@ def main():
                                                                   "workloads; spd_stack times inverse roots only"}))
             return
         run_spd(args)
+        return
+    if args.config == "evd_stack":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the optimizer-step "
+                                                                  "workloads; evd_stack times inverse roots only"}))
+            return
+        run_evd(args)
         return
     cfg = CONFIGS[args.config]
     if args.impl == "reference":

@@ -77,6 +77,16 @@ typedef int32_t shp_status;
 
 /* Bits of the per-matrix status written by shampoo_inv_root. */
 #define SHP_ROOT_NONFINITE 1
+#define SHP_ROOT_UNCONVERGED 2 /* shampoo_inv_root_evd: sweep limit reached */
+
+/* Dampening heuristics of shampoo_inv_root_evd ([DASH] B.1, B.2). */
+#define SHP_EVD_CORRECTED 0
+#define SHP_EVD_SHIFTED_RELU 1
+#define SHP_EVD_ABS_ADD 2
+#define SHP_EVD_SHMP 3
+
+/* Largest side shampoo_inv_root_evd accepts (shared-memory resident). */
+#define SHP_EVD_MAX_N 128
 
 /* Columns of the block table (shampoo_plan_tables). */
 #define SHP_BLOCK_FIELDS 13
@@ -264,6 +274,34 @@ SHP_API size_t shampoo_inv_root_warm_workspace_bytes(int32_t count, int32_t n, i
 SHP_API shp_status shampoo_inv_root_warm(const float* A, const float* X0, int32_t count, int32_t n, float eps,
                                          int32_t p, int32_t iters, int32_t dtype, float* X_out,
                                          int32_t* status_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Inverse p-th roots by eigendecomposition   ([DASH] §3 (EVD, the
+ * reference method), B.1 regularisation for EVD, B.2 dampening heuristics)
+ *   mu, Q = eig(L + eps I) (L symmetrised as (L + L^T)/2), lambda = mu - eps
+ *   (the corrected spectrum), X = Q diag(f) Q^T with, by heuristic:
+ *     SHP_EVD_CORRECTED     f = (max(lambda, 0) + eps)^(-1/p)
+ *     SHP_EVD_SHIFTED_RELU  f = (lambda - eps)^(-1/p) where lambda > eps,
+ *                           else 0 (a rank-r_eps inverse)
+ *     SHP_EVD_ABS_ADD       f = (|lambda| + eps)^(-1/p)
+ *     SHP_EVD_SHMP          f = (mu - min(min_i mu_i, 0) + eps)^(-1/p), the
+ *                           Distributed Shampoo adjustment (eps added twice)
+ * The eigensolver is cyclic two-sided Jacobi, one CTA per matrix held in
+ * shared memory (the matrix rotated in float64, the eigenvectors
+ * accumulated in float32), until a sweep leaves every off-diagonal
+ * entry below 2^-21 sqrt(|a_pp a_qq|) (at most 40 sweeps; otherwise the
+ * matrix's status gets SHP_ROOT_UNCONVERGED).
+ * A: device (count, n, n) float32 row-major; X_out: same shape (may be A);
+ * eig_out: NULL or device (count, n) float32, lambda ascending per matrix;
+ * status_out: device [count] int32, SHP_ROOT_* bits in bits 0-7 and the
+ *   number of sweeps taken in bits 8-15 (the final sweep, which rotates
+ *   nothing, included).
+ * Sizes: 1 <= n <= SHP_EVD_MAX_N (any n), count >= 1; p in {2, 4, 8}.
+ * No workspace.  Errors (nothing enqueued): SHP_ERR_INVALID_ARG (NULL
+ * pointer, bad heuristic, eps < 0 or not finite), SHP_ERR_SHAPE (n, count),
+ * SHP_ERR_UNSUPPORTED (other p), SHP_ERR_CUDA (launch failure). */
+SHP_API shp_status shampoo_inv_root_evd(const float* A, int32_t count, int32_t n, float eps, int32_t p,
+                                        int32_t heuristic, float* X_out, float* eig_out, int32_t* status_out,
+                                        void* stream);
 
 /* ---------------------------------------------------------------------
  * a7  Two-sided preconditioning   ([DASH] §2)

@@ -28,7 +28,7 @@ EXPORTS = [
     "shampoo_plan_bind", "shampoo_stack_blocks",
     "shampoo_update_stats_workspace_bytes", "shampoo_update_stats",
     "shampoo_inv_root_workspace_bytes", "shampoo_inv_root", "shampoo_inv_root_static",
-    "shampoo_inv_root_warm_workspace_bytes", "shampoo_inv_root_warm",
+    "shampoo_inv_root_warm_workspace_bytes", "shampoo_inv_root_warm", "shampoo_inv_root_evd",
     "shampoo_precondition_workspace_bytes", "shampoo_precondition",
     "shampoo_graft_step_workspace_bytes", "shampoo_graft_step",
 ]
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         "shampoo_inv_root_warm_workspace_bytes": (c_size_t, [c_int32] * 3),
         "shampoo_inv_root_warm": (c_int32, [c_void_p, c_void_p, c_int32, c_int32, c_float, c_int32, c_int32,
                                             c_int32, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+        "shampoo_inv_root_evd": (c_int32, [c_void_p, c_int32, c_int32, c_float, c_int32, c_int32, c_void_p,
+                                           c_void_p, c_void_p, c_void_p]),
         "shampoo_precondition_workspace_bytes": (c_size_t, [c_void_p, c_int32]),
         "shampoo_precondition": (c_int32, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), c_void_p, c_int32,
                                            c_void_p, c_size_t, c_void_p]),
@@ -247,6 +249,26 @@ def inv_root_warm(A, X0, eps: float, iters: int = 3, dtype="fp32", p: int = 4, o
                                        _enum(DTYPES, dtype), _ptr(X), _ptr(st), _ptr(workspace), workspace.numel(),
                                        _stream(stream)), "shampoo_inv_root_warm")
     return X, st
+
+
+EVD_HEURISTICS = {"corrected": 0, "shifted_relu": 1, "abs_add": 2, "shmp": 3}
+EVD_MAX_N = 128
+
+
+def inv_root_evd(A, eps: float, heuristic="corrected", p: int = 4, out=None, eig_out=None, status_out=None,
+                 want_eig: bool = False, stream=None):
+    """Inverse p-th roots of a (count, n, n) float32 CUDA stack by Jacobi
+    eigendecomposition with a dampening heuristic; returns (X, eigenvalues
+    of L ascending or None, status).  ``out`` may be A."""
+    import torch
+    count, n = int(A.shape[0]), int(A.shape[1])
+    X = out if out is not None else torch.empty_like(A)
+    ev = eig_out if eig_out is not None else (
+        torch.empty((count, n), dtype=torch.float32, device=A.device) if want_eig else None)
+    st = status_out if status_out is not None else torch.empty(count, dtype=torch.int32, device=A.device)
+    _check(lib().shampoo_inv_root_evd(_ptr(A), count, n, float(eps), int(p), _enum(EVD_HEURISTICS, heuristic),
+                                      _ptr(X), _ptr(ev), _ptr(st), _stream(stream)), "shampoo_inv_root_evd")
+    return X, ev, st
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libshampoo.so")
-SOURCES = ["api.cu", "gemm.cu", "kernels.cu", "step_kernels.cu", "static_scratch.cu"]
+SOURCES = ["api.cu", "gemm.cu", "kernels.cu", "step_kernels.cu", "static_scratch.cu", "evd.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]

@@ -900,6 +900,20 @@ shp_status shampoo_inv_root_warm(const float* A, const float* X0, int32_t count,
   return run_cn_warm(A, X0, count, n, eps, iters, p, (Prec)dtype, r, X_out, status_out, st);
 }
 
+shp_status shampoo_inv_root_evd(const float* A, int32_t count, int32_t n, float eps, int32_t p, int32_t heuristic,
+                                float* X_out, float* eig_out, int32_t* status_out, void* stream) {
+  if (n < 1 || n > SHP_EVD_MAX_N) return fail(SHP_ERR_SHAPE, "n %d: need 1 <= n <= %d", n, SHP_EVD_MAX_N);
+  if (count < 1) return fail(SHP_ERR_SHAPE, "count %d must be >= 1", count);
+  if (p != 2 && p != 4 && p != 8) return fail(SHP_ERR_UNSUPPORTED, "root power p must be 2, 4 or 8");
+  if (heuristic < SHP_EVD_CORRECTED || heuristic > SHP_EVD_SHMP)
+    return fail(SHP_ERR_INVALID_ARG, "bad heuristic %d", heuristic);
+  if (!A || !X_out || !status_out) return fail(SHP_ERR_INVALID_ARG, "A, X_out and status_out must be non-NULL");
+  if (!std::isfinite(eps) || eps < 0.f) return fail(SHP_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  cudaError_t e = launch_evd_root(A, count, n, eps, p, heuristic, X_out, eig_out, status_out, as_stream(stream));
+  if (e != cudaSuccess) return fail(SHP_ERR_CUDA, "EVD launch: %s", cudaGetErrorString(e));
+  return SHP_OK;
+}
+
 // ---- precondition ----------------------------------------------------------
 
 struct PrecBufs {

@@ -139,6 +139,11 @@ cudaError_t launch_pi_rayleigh(const float* W, const void* vt_h16, int n, int v,
 
 cudaError_t launch_zero_i32(int* p, size_t n, cudaStream_t stream);
 
+// Inverse roots by Jacobi eigendecomposition, one CTA per matrix (evd.cu).
+size_t evd_smem_bytes(int n);
+cudaError_t launch_evd_root(const float* A, int count, int n, float eps, int p, int heuristic, float* X, float* eig,
+                            int* status, cudaStream_t stream);
+
 // Host-side count of kernel launches issued by the library.
 void count_launch();
 unsigned long long launch_total();

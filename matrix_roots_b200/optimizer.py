@@ -4,6 +4,8 @@ With ``precond_every`` = f > 1 the roots are recomputed only on steps 1,
 1 + f, ... and the stale roots precondition the steps between ("3D-Shampoo
 optimizer" README, Hyperparameters: preconditioning_compute_steps; DASH §1,
 roots every 10-100 steps); the statistics are updated every step.
+Method "evd" takes the roots from shampoo_inv_root_evd (blocks up to 128)
+with the dampening heuristic ``evd_heuristic`` (DASH B.1-B.2).
 
 ``BlockedShampoo`` owns the device state (gradient / factor / root /
 direction stacks, graft moments and one shared workspace) and calls, in
@@ -46,6 +48,7 @@ class ShampooConfig:
     root_p: int = 4             # inverse p-th roots, p in (2, 4, 8)
     graph: bool = False         # replay the launches before the graft step as a CUDA graph
     layerwise: bool = False     # stack per layer instead of across all layers
+    evd_heuristic: str = "corrected"  # method "evd": corrected, shifted_relu, abs_add or shmp
 
 
 class BlockedShampoo:
@@ -77,7 +80,7 @@ class BlockedShampoo:
              B.precondition_workspace_bytes(self.plan, cfg.precond_dtype),
              B.graft_step_workspace_bytes(self.plan)]
             + [B.inv_root_workspace_bytes(int(c), int(n), cfg.method, cfg.dtype, cfg.scaling, cfg.pi_vectors)
-               for n, c in t["f_buckets"]])
+               for n, c in (t["f_buckets"] if cfg.method != "evd" else [])])
         self.workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
         self.t = 0
         self._graphs = {}       # (fresh roots?, gradient addresses) -> (CUDAGraph, library launches in it)
@@ -90,6 +93,10 @@ class BlockedShampoo:
         B.stack_blocks(self.plan, G, self.g_stacks, stream)
         B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
         for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
+            if c.method == "evd":
+                B.inv_root_evd(self.factors[fb], c.eps, c.evd_heuristic, c.root_p, out=self.roots[fb],
+                               status_out=self.status[fb], stream=stream)
+                continue
             B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, c.root_p, c.pi_vectors, c.pi_iters,
                        self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,

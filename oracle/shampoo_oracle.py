@@ -667,8 +667,10 @@ class ShampooState:
         self.roots = None  # the last computed inverse roots, per factor bucket
 
 
-def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec):
-    """Inverse fourth roots of every factor of the state (a3-a6)."""
+def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec,
+                  evd_heuristic="corrected"):
+    """Inverse fourth roots of every factor of the state (a3-a6; EVD with
+    the heuristic of reading R15)."""
     roots = [np.empty_like(f) for f in state.factors]
     for fb, stack in enumerate(state.factors):
         for i in range(stack.shape[0]):
@@ -681,7 +683,10 @@ def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scale
                 s = power_iteration_scale(Lf, 0.0 if method == "cheb" else eps, pi_starts, pi_iters)
             if scales_out is not None:
                 scales_out[(fb, i)] = s
-            roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay, prec=prec)
+            if method == "evd" and evd_heuristic != "corrected":
+                roots[fb][i] = evd_inv_root(Lf, eps, evd_heuristic)
+            else:
+                roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay, prec=prec)
     return roots
 
 
@@ -689,7 +694,7 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
                  method: str, iters: int, scaling: str, graft: str, lr: float,
                  beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
                  wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
-                 replay: bool = True, prec=None, precond_every: int = 1):
+                 replay: bool = True, prec=None, precond_every: int = 1, evd_heuristic: str = "corrected"):
     """One optimizer step over all layers; returns the new weights.
 
     ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
@@ -712,7 +717,8 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
     if state.roots is not None and (state.step - 1) % max(int(precond_every), 1) != 0:
         roots = state.roots
     else:
-        roots = compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec)
+        roots = compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec,
+                              evd_heuristic)
         state.roots = roots
     d_st = [np.empty_like(g) for g in g_st]
     for b in plan["blocks"]:

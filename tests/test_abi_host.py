@@ -195,3 +195,27 @@ def test_inv_root_warm_rejects_before_enqueue(over, code):
 def test_inv_root_warm_workspace_is_the_cn_workspace():
     assert B.inv_root_warm_workspace_bytes(8, 64) == B.inv_root_workspace_bytes(8, 64, "cn", "fp32")
     assert B.inv_root_warm_workspace_bytes(8, 6) == 0
+
+
+def _call_evd(**over):
+    L = B.lib()
+    args = dict(A=0x1000, count=4, n=64, eps=1e-6, p=4, heuristic=0, X=0x2000, eig=0, status=0x4000, stream=0)
+    args.update(over)
+    return L.shampoo_inv_root_evd(args["A"], args["count"], args["n"], args["eps"], args["p"], args["heuristic"],
+                                  args["X"], args["eig"], args["status"], args["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(A=0), B.SHP_ERR_INVALID_ARG),
+    (dict(X=0), B.SHP_ERR_INVALID_ARG),
+    (dict(status=0), B.SHP_ERR_INVALID_ARG),
+    (dict(heuristic=4), B.SHP_ERR_INVALID_ARG),
+    (dict(heuristic=-1), B.SHP_ERR_INVALID_ARG),
+    (dict(eps=float("inf")), B.SHP_ERR_INVALID_ARG),
+    (dict(n=0), B.SHP_ERR_SHAPE),
+    (dict(n=129), B.SHP_ERR_SHAPE),
+    (dict(count=0), B.SHP_ERR_SHAPE),
+    (dict(p=3), B.SHP_ERR_UNSUPPORTED),
+])
+def test_inv_root_evd_rejects_before_enqueue(over, code):
+    assert _call_evd(**over) == code

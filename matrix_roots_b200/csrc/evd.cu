@@ -9,8 +9,10 @@
 // n + 1, so row and column sweeps are both free of bank conflicts; that
 // bounds n at 128 (128 x 129 x (8 + 4) B = 198 KB).  The eigensolver is
 // two-sided cyclic Jacobi in the round-robin pair order: each round rotates
-// n/2 disjoint (p, q) planes at once -- rows first, then columns and V -- so
-// one CTA keeps all its warps busy on independent rotations.  A plane is
+// n/2 disjoint (p, q) planes at once, one warp per plane: the warp works
+// out its plane's rotation and rotates the two rows, and after a barrier the
+// same warps rotate the two columns of A and of V (two barriers a round).
+// A plane is
 // rotated only while its off-diagonal entry is above 2^-21 sqrt(|a_pp
 // a_qq|); a sweep without rotations ends the solve.  Then X = V diag(f(mu))
 // V^T with f the chosen heuristic, written row-major in float32.
@@ -31,6 +33,7 @@ namespace shp {
 namespace {
 
 constexpr int kEvdThreads = 512;
+constexpr int kEvdWarps = kEvdThreads / 32;
 constexpr int kEvdMaxSweeps = 40;
 constexpr float kRelTol = 4.76837158e-7f;  // 2^-21
 
@@ -61,6 +64,7 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
   __shared__ double mu_min_s;
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int ld = n + 1;
   double* a = smem;
   float* v = reinterpret_cast<float*>(smem + n * ld);
@@ -95,8 +99,11 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
   int sweeps = 0;
   for (; sweeps < kEvdMaxSweeps && !converged; ++sweeps) {
     for (int round = 0; round < m - 1; ++round) {
-      if (tid < half) {
-        const int k = tid;
+      // Rotation angles and rows: warp w owns pairs w, w + 16, ...; its
+      // lanes read the pivot entries (broadcast), agree on the rotation,
+      // then rotate rows p and q, 32 columns at a time.  No other warp
+      // touches those two rows in this phase.
+      for (int k = warp; k < half; k += kEvdWarps) {
         int P = k == 0 ? 0 : 1 + (k - 1 + round) % (m - 1);
         int Q = 1 + (m - 2 - k + round) % (m - 1);
         if (P > Q) {
@@ -112,60 +119,60 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
           if (apq != 0.0 && fabs(apq) > kRelTol * sqrt(fabs(app) * fabs(aqq))) {
             // tan of the angle that zeroes a_pq, the smaller root (|t| <= 1)
             const double th = (aqq - app) / (2.0 * apq);
-            t = copysign(1.0, th) / (fabs(th) + hypot(1.0, th));
+            const double ath = fabs(th);
+            t = ath > 1e150 ? 0.5 / th : copysign(1.0, th) / (ath + sqrt(1.0 + th * th));
             const double c = 1.0 / sqrt(1.0 + t * t);
             s = t * c;
             tau2 = s / (1.0 + c);
-            rotated = 1;
           }
         }
-        pr_p[k] = P;
-        pr_q[k] = Q;
-        pr_s[k] = s;
-        pr_tau[k] = tau2;
-        pr_t[k] = t;
-        pr_app[k] = app;
-        pr_aqq[k] = aqq;
-        pr_apq[k] = apq;
-      }
-      __syncthreads();
-      // rows p, q <- J^T rows
-      for (int i = tid; i < half * n; i += blockDim.x) {
-        const int k = i / n, j = i - k * n;
-        const double s = pr_s[k];
+        if (lane == 0) {
+          pr_p[k] = P;
+          pr_q[k] = Q;
+          pr_s[k] = s;
+          pr_tau[k] = tau2;
+          pr_t[k] = t;
+          pr_app[k] = app;
+          pr_aqq[k] = aqq;
+          pr_apq[k] = apq;
+          if (s != 0.0) rotated = 1;
+        }
+        __syncwarp();  // every lane has read the pivot entries
         if (s == 0.0) continue;
-        const double tau2 = pr_tau[k];
-        double* rp = a + pr_p[k] * ld;
-        double* rq = a + pr_q[k] * ld;
-        const double x = rp[j], y = rq[j];
-        rp[j] = x - s * (y + tau2 * x);
-        rq[j] = y + s * (x - tau2 * y);
+        double* rp = a + P * ld;
+        double* rq = a + Q * ld;
+        for (int j = lane; j < n; j += 32) {
+          const double x = rp[j], y = rq[j];
+          rp[j] = x - s * (y + tau2 * x);
+          rq[j] = y + s * (x - tau2 * y);
+        }
       }
       __syncthreads();
       // columns p, q of A and V <- . J; the 2 x 2 pivot block set exactly
-      for (int i = tid; i < half * n; i += blockDim.x) {
-        const int k = i / n, r = i - k * n;
+      for (int k = warp; k < half; k += kEvdWarps) {
         const double s = pr_s[k];
         if (s == 0.0) continue;
         const double tau2 = pr_tau[k];
         const int P = pr_p[k], Q = pr_q[k];
-        double* ar = a + r * ld;
-        const double x = ar[P], y = ar[Q];
-        double nx = x - s * (y + tau2 * x), ny = y + s * (x - tau2 * y);
-        if (r == P) {
-          nx = pr_app[k] - pr_t[k] * pr_apq[k];
-          ny = 0.0;
-        } else if (r == Q) {
-          nx = 0.0;
-          ny = pr_aqq[k] + pr_t[k] * pr_apq[k];
-        }
-        ar[P] = nx;
-        ar[Q] = ny;
         const float sf = (float)s, tf = (float)tau2;
-        float* vr = v + r * ld;
-        const float vx = vr[P], vy = vr[Q];
-        vr[P] = vx - sf * (vy + tf * vx);
-        vr[Q] = vy + sf * (vx - tf * vy);
+        for (int r = lane; r < n; r += 32) {
+          double* ar = a + r * ld;
+          const double x = ar[P], y = ar[Q];
+          double nx = x - s * (y + tau2 * x), ny = y + s * (x - tau2 * y);
+          if (r == P) {
+            nx = pr_app[k] - pr_t[k] * pr_apq[k];
+            ny = 0.0;
+          } else if (r == Q) {
+            nx = 0.0;
+            ny = pr_aqq[k] + pr_t[k] * pr_apq[k];
+          }
+          ar[P] = nx;
+          ar[Q] = ny;
+          float* vr = v + r * ld;
+          const float vx = vr[P], vy = vr[Q];
+          vr[P] = vx - sf * (vy + tf * vx);
+          vr[Q] = vy + sf * (vx - tf * vy);
+        }
       }
       __syncthreads();
     }

@@ -49,6 +49,16 @@ R12 Root power p: p in {2, 4, 8} ([Notes] "Spreading the preconditioners":
 R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
     Hyperparameters: preconditioning_compute_steps; [DASH] §1).
+R16 One-sided layers ([Notes] "Roots on idle CPUs": embedding and softmax
+    layers, and layers too large for a right factor, are preconditioned on
+    one side only, L^{-1/2} G, the alpha = 1 split of the Kronecker bound):
+    such a layer keeps only left factors; its gradient and factor stacks are
+    separate from the two-sided ones (bucket keys carry the side); its
+    roots are inverse square roots, D = X_L G.  A layer whose large side is
+    its rows is passed transposed by the caller.
+R17 Shape interpretation ([DASH] D: a ViT embedding (E, 3, 16, 16) becomes
+    (E, 768)): a parameter of rank > 2 is preconditioned as the matrix
+    (first dimension, product of the others); rank 1 and 0 are not.
 R15 EVD roots with the dampening heuristics of [DASH] B.1-B.2: the
     eigendecomposition is taken of L + eps I, mu = its eigenvalues, and
     lambda = mu - eps (the corrected spectrum).  corrected: (max(lambda, 0)
@@ -75,7 +85,7 @@ import numpy as np
 
 __all__ = [
     "BLOCK_FIELDS", "split_dim", "plan_blocks", "stack_gradients", "unstack_directions",
-    "update_stats", "spd_power", "inv_root_exact", "EVD_HEURISTICS", "evd_root_factors", "evd_inv_root",
+    "matrix_shape", "update_stats", "spd_power", "inv_root_exact", "EVD_HEURISTICS", "evd_root_factors", "evd_inv_root",
     "frobenius_scale", "power_iteration_scale",
     "ndb_matrix", "ndb_calls", "ndb_inv_root", "ndb_scalar", "ndb_inv_root_replay",
     "cn_matrix", "cn_inv_root", "cn_inv_root_warm", "cn_scalar", "cn_inv_root_replay",
@@ -113,35 +123,42 @@ def split_dim(d: int, block_size: int) -> list[int]:
     return sizes
 
 
-def plan_blocks(shapes, block_size: int, layerwise: bool = False) -> dict:
+def plan_blocks(shapes, block_size: int, layerwise: bool = False, left_only=None) -> dict:
     """Partition every layer into blocks and assign them to stacks.
 
     Returns int32 tables:
       blocks    (n_blocks, 13) with the columns of ``BLOCK_FIELDS``;
       g_buckets (n_g, 3)  rows, cols, count of each gradient-block stack;
-      f_buckets (n_f, 2)  n, count of each preconditioner-factor stack.
+      f_buckets (n_f, 2)  n, count of each preconditioner-factor stack;
+      f_sides   (n_f,)    0: factors of two-sided blocks, 1: left factors of
+                          one-sided blocks (reading R16).
     Gradient blocks are bucketed by (rows, cols), factors by n ([DASH] §4);
     the order inside buckets is reading R1.  ``layerwise`` keys the buckets
     by layer as well ([DASH] §4: DASH-LAYERWISE stacks per layer, DASH-GPU
-    across all layers of a GPU).
+    across all layers of a GPU).  ``left_only[i]`` true makes layer i
+    one-sided: its blocks get no right factor (fields -1) and both its
+    buckets are keyed by the side too.
     """
     blocks = []
     g_key_to_id: dict = {}
     g_counts: list = []
     f_key_to_id: dict = {}
     f_counts: list = []
+    f_sides: list = []
 
-    def f_slot(n, li):
-        key = (li, n) if layerwise else n
+    def f_slot(n, li, side):
+        key = (li, n, side) if layerwise else (n, side)
         if key not in f_key_to_id:
             f_key_to_id[key] = len(f_counts)
             f_counts.append([n, 0])
+            f_sides.append(side)
         b = f_key_to_id[key]
         idx = f_counts[b][1]
         f_counts[b][1] += 1
         return b, idx
 
     for li, (m, n) in enumerate(shapes):
+        side = 1 if left_only is not None and left_only[li] else 0
         rs = split_dim(int(m), block_size)
         cs = split_dim(int(n), block_size)
         layer_blocks = []
@@ -149,7 +166,7 @@ def plan_blocks(shapes, block_size: int, layerwise: bool = False) -> dict:
         for br, r in enumerate(rs):
             col0 = 0
             for bc, c in enumerate(cs):
-                key = (li, r, c) if layerwise else (r, c)
+                key = (li, r, c, side) if layerwise else (r, c, side)
                 if key not in g_key_to_id:
                     g_key_to_id[key] = len(g_counts)
                     g_counts.append([r, c, 0])
@@ -160,15 +177,26 @@ def plan_blocks(shapes, block_size: int, layerwise: bool = False) -> dict:
                 col0 += c
             row0 += r
         for blk in layer_blocks:          # all left factors of the layer, row-major
-            blk[9], blk[10] = f_slot(blk[5], li)
-        for blk in layer_blocks:          # then all right factors, row-major
-            blk[11], blk[12] = f_slot(blk[6], li)
+            blk[9], blk[10] = f_slot(blk[5], li, side)
+        if not side:
+            for blk in layer_blocks:      # then all right factors, row-major
+                blk[11], blk[12] = f_slot(blk[6], li, side)
         blocks += layer_blocks
     return {
         "blocks": np.asarray(blocks, dtype=np.int32).reshape(-1, len(BLOCK_FIELDS)),
         "g_buckets": np.asarray(g_counts, dtype=np.int32).reshape(-1, 3),
         "f_buckets": np.asarray(f_counts, dtype=np.int32).reshape(-1, 2),
+        "f_sides": np.asarray(f_sides, dtype=np.int32),
     }
+
+
+def matrix_shape(shape):
+    """The matrix a parameter is preconditioned as (reading R17): rank 2 as
+    is, rank > 2 as (first dimension, product of the rest), else None."""
+    shape = tuple(int(x) for x in shape)
+    if len(shape) < 2:
+        return None
+    return (shape[0], int(np.prod(shape[1:])))
 
 
 def stack_gradients(plan: dict, grads) -> list[np.ndarray]:
@@ -656,9 +684,9 @@ def graft_update(W, G, D, m, v, kind: str, lr: float, beta1: float, beta2: float
 class ShampooState:
     """Optimizer state of the oracle: factor stacks and graft moments."""
 
-    def __init__(self, shapes, block_size: int, graft: str):
+    def __init__(self, shapes, block_size: int, graft: str, left_only=None):
         self.shapes = [tuple(int(x) for x in s) for s in shapes]
-        self.plan = plan_blocks(self.shapes, block_size)
+        self.plan = plan_blocks(self.shapes, block_size, left_only=left_only)
         self.factors = [np.zeros((int(c), int(n), int(n))) for (n, c) in self.plan["f_buckets"]]
         need = graft in ("adam", "adagrad")
         self.m = [np.zeros(s) for s in self.shapes] if graft == "adam" else [None] * len(self.shapes)
@@ -670,9 +698,11 @@ class ShampooState:
 def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scales_out, replay, prec,
                   evd_heuristic="corrected"):
     """Inverse fourth roots of every factor of the state (a3-a6; EVD with
-    the heuristic of reading R15)."""
+    the heuristic of reading R15); inverse square roots for the factors of
+    one-sided layers (reading R16)."""
     roots = [np.empty_like(f) for f in state.factors]
     for fb, stack in enumerate(state.factors):
+        p = 2 if state.plan["f_sides"][fb] else 4
         for i in range(stack.shape[0]):
             Lf = stack[i]
             if method == "evd":
@@ -684,9 +714,9 @@ def compute_roots(state, eps, method, iters, scaling, pi_starts, pi_iters, scale
             if scales_out is not None:
                 scales_out[(fb, i)] = s
             if method == "evd" and evd_heuristic != "corrected":
-                roots[fb][i] = evd_inv_root(Lf, eps, evd_heuristic)
+                roots[fb][i] = evd_inv_root(Lf, eps, evd_heuristic, p)
             else:
-                roots[fb][i] = inv_root(Lf, eps, method, iters, s, replay=replay, prec=prec)
+                roots[fb][i] = inv_root(Lf, eps, method, iters, s, p=p, replay=replay, prec=prec)
     return roots
 
 
@@ -710,6 +740,10 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
     g_st = stack_gradients(plan, grads)
     for b in plan["blocks"]:
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
+        if rb < 0:  # one-sided layer: left statistics only (reading R16)
+            g = np.asarray(g_st[gb][gi], dtype=np.float64)
+            state.factors[lb][lix] = beta2 * state.factors[lb][lix] + alpha * (g @ g.T)
+            continue
         state.factors[lb][lix], state.factors[rb][rix] = update_stats(
             g_st[gb][gi], state.factors[lb][lix], state.factors[rb][rix], beta2, alpha)
     if prec is not None:  # the arithmetic model also stores the statistics in float32
@@ -723,6 +757,9 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
     d_st = [np.empty_like(g) for g in g_st]
     for b in plan["blocks"]:
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
+        if rb < 0:
+            d_st[gb][gi] = np.asarray(roots[lb][lix], np.float64) @ np.asarray(g_st[gb][gi], np.float64)
+            continue
         d_st[gb][gi] = precondition(roots[lb][lix], g_st[gb][gi], roots[rb][rix])
     D = unstack_directions(plan, d_st, state.shapes)
     newW = []

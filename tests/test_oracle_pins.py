@@ -701,3 +701,46 @@ def test_evd_corrected_is_the_exact_root_and_shifted_relu_kills_the_null_space()
     w, U = np.linalg.eigh(L)
     U5, w5 = U[:, -5:], w[-5:]
     assert O.rel_fro(U5.T @ X @ U5, np.diag((w5 - 1e-3) ** -0.25)) < 1e-9
+
+
+# ---- one-sided layers and shape interpretation (readings R16, R17) ----------
+
+def test_plan_one_sided_layers():
+    """A one-sided layer keeps left factors only, in stacks of its own."""
+    shapes = [(128, 96), (128, 96), (64, 64)]
+    pl = O.plan_blocks(shapes, 64, left_only=[False, True, False])
+    blk = pl["blocks"]
+    one = blk[blk[:, 0] == 1]
+    assert (one[:, 11] == -1).all() and (one[:, 12] == -1).all()
+    assert (blk[blk[:, 0] != 1][:, 11] >= 0).all()
+    # no stack mixes sides
+    assert set(one[:, 7]).isdisjoint(set(blk[blk[:, 0] != 1][:, 7]))
+    assert set(one[:, 9]).isdisjoint(set(blk[blk[:, 0] != 1][:, 9]))
+    assert all(pl["f_sides"][f] == 1 for f in one[:, 9])
+    # with no one-sided layer the tables are the two-sided plan's
+    a, b = O.plan_blocks(shapes, 64), O.plan_blocks(shapes, 64, left_only=[False] * 3)
+    for k in ("blocks", "g_buckets", "f_buckets", "f_sides"):
+        assert np.array_equal(a[k], b[k])
+    assert (a["f_sides"] == 0).all()
+
+
+def test_one_sided_step_is_the_svd_closed_form():
+    """One step, beta2 = 1, one block: L = G G^T, X_L = (L + eps I)^{-1/2},
+    so D = U diag(s / sqrt(s^2 + eps)) V^T from the SVD G = U diag(s) V^T,
+    and with no graft W = -lr D."""
+    rng = np.random.default_rng(31)
+    G = rng.standard_normal((24, 40))
+    st = O.ShampooState([(24, 40)], 0, "none", left_only=[True])
+    W = O.shampoo_step(st, [np.zeros((24, 40))], [G], beta2=1.0, alpha=1.0, eps=1e-2, method="evd",
+                       iters=0, scaling="frobenius", graft="none", lr=0.5)
+    U, sv, Vt = np.linalg.svd(G, full_matrices=False)
+    D = (U * (sv / np.sqrt(sv ** 2 + 1e-2))) @ Vt
+    assert O.rel_fro(W[0], -0.5 * D) < 1e-10
+    assert len(st.factors) == 1 and st.factors[0].shape == (1, 24, 24)
+
+
+def test_matrix_shape_merges_trailing_dimensions():
+    assert O.matrix_shape((384, 3, 16, 16)) == (384, 768)
+    assert O.matrix_shape((512, 5, 5, 64)) == (512, 1600)
+    assert O.matrix_shape((7, 9)) == (7, 9)
+    assert O.matrix_shape((10,)) is None and O.matrix_shape(()) is None

@@ -134,15 +134,30 @@ SHP_API shp_status shampoo_device_error(int32_t* out);
 SHP_API shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
                                shp_plan** plan_out);
 
-/* shampoo_plan_create with flags.  SHP_PLAN_LAYERWISE stacks per layer:
- * gradient buckets are keyed by (layer, rows, cols) and factor buckets by
- * (layer, n), the "layerwise" stacking the DASH paper compares with its
- * GPU-level stacking (§4 Blocking Strategy); the order inside a bucket is
- * unchanged.  flags 0 is shampoo_plan_create; unknown bits return
- * SHP_ERR_INVALID_ARG.  The paper has no flag: it names the two variants. */
+/* shampoo_plan_create with one-sided layers and flags.
+ * left_only: NULL, or host [n_layers]; nonzero makes that layer one-sided
+ *   ([Notes] "Roots on idle CPUs": embedding, softmax and very large
+ *   layers are preconditioned on one side only, L^(-1/2) G): its blocks get
+ *   left factors only (r_bucket = r_index = -1), and its gradient and factor
+ *   buckets are keyed by that side as well, so no stack mixes one- and
+ *   two-sided blocks.  shampoo_update_stats then updates only L for them,
+ *   shampoo_precondition computes D = X_L G, and the caller takes inverse
+ *   square roots (p = 2) of the buckets shampoo_plan_factor_sides marks 1.
+ *   A layer whose large side is its rows is passed transposed.
+ * flags: SHP_PLAN_LAYERWISE stacks per layer: gradient buckets are keyed by
+ *   (layer, rows, cols) and factor buckets by (layer, n), the "layerwise"
+ *   stacking the DASH paper compares with its GPU-level stacking (§4
+ *   Blocking Strategy); the order inside a bucket is unchanged.  The paper
+ *   has no flag: it names the two variants.  Unknown bits return
+ *   SHP_ERR_INVALID_ARG.
+ * NULL left_only with flags 0 is shampoo_plan_create. */
 #define SHP_PLAN_LAYERWISE 1
-SHP_API shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int32_t n_layers,
-                                          int32_t block_size, int32_t flags, shp_plan** plan_out);
+SHP_API shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, const int32_t* left_only,
+                                          int32_t n_layers, int32_t block_size, int32_t flags, shp_plan** plan_out);
+
+/* Side of every factor bucket: host [n_fbuckets], 0 for factors of
+ * two-sided blocks, 1 for the left factors of one-sided blocks. */
+SHP_API shp_status shampoo_plan_factor_sides(const shp_plan* plan, int32_t* sides);
 SHP_API void shampoo_plan_destroy(shp_plan* plan);
 
 /* Table sizes: number of blocks, of gradient buckets, of factor buckets, and

@@ -24,7 +24,7 @@ BLOCK_FIELDS = 13
 EXPORTS = [
     "shampoo_last_error", "shampoo_version", "shampoo_launch_count", "shampoo_device_error",
     "shampoo_plan_create", "shampoo_plan_create_ex", "shampoo_plan_destroy", "shampoo_plan_sizes",
-    "shampoo_plan_tables",
+    "shampoo_plan_tables", "shampoo_plan_factor_sides",
     "shampoo_plan_bind", "shampoo_stack_blocks",
     "shampoo_update_stats_workspace_bytes", "shampoo_update_stats",
     "shampoo_inv_root_workspace_bytes", "shampoo_inv_root", "shampoo_inv_root_static",
@@ -59,7 +59,9 @@ def lib() -> ctypes.CDLL:
         "shampoo_launch_count": (ctypes.c_uint64, []),
         "shampoo_device_error": (c_int32, [P(c_int32)]),
         "shampoo_plan_create": (c_int32, [P(c_int32), P(c_int32), c_int32, c_int32, P(c_void_p)]),
-        "shampoo_plan_create_ex": (c_int32, [P(c_int32), P(c_int32), c_int32, c_int32, c_int32, P(c_void_p)]),
+        "shampoo_plan_create_ex": (c_int32, [P(c_int32), P(c_int32), P(c_int32), c_int32, c_int32, c_int32,
+                                             P(c_void_p)]),
+        "shampoo_plan_factor_sides": (c_int32, [c_void_p, P(c_int32)]),
         "shampoo_plan_destroy": (None, [c_void_p]),
         "shampoo_plan_sizes": (c_int32, [c_void_p, P(c_int32), P(c_int32), P(c_int32), P(c_size_t)]),
         "shampoo_plan_tables": (c_int32, [c_void_p, P(c_int32), P(c_int32), P(c_int32)]),
@@ -147,14 +149,20 @@ def device_error() -> int:
 
 class Plan:
     """Host block plan (shampoo_plan_create_ex) plus its bound device tables;
-    ``layerwise`` stacks per layer (SHP_PLAN_LAYERWISE)."""
+    ``layerwise`` stacks per layer (SHP_PLAN_LAYERWISE); ``left_only`` (one
+    flag per layer, or None) makes layers one-sided."""
 
-    def __init__(self, shapes, block_size: int, layerwise: bool = False):
+    def __init__(self, shapes, block_size: int, layerwise: bool = False, left_only=None):
         self.shapes = [(int(m), int(n)) for (m, n) in shapes]
         rows = (c_int32 * len(self.shapes))(*[m for m, _ in self.shapes])
         cols = (c_int32 * len(self.shapes))(*[n for _, n in self.shapes])
+        lo = None
+        if left_only is not None:
+            if len(left_only) != len(self.shapes):
+                raise ValueError("left_only needs one flag per layer")
+            lo = (c_int32 * len(self.shapes))(*[1 if x else 0 for x in left_only])
         h = c_void_p()
-        _check(lib().shampoo_plan_create_ex(rows, cols, len(self.shapes), int(block_size), 1 if layerwise else 0,
+        _check(lib().shampoo_plan_create_ex(rows, cols, lo, len(self.shapes), int(block_size), 1 if layerwise else 0,
                                             ctypes.byref(h)), "shampoo_plan_create_ex")
         self.handle = h
         nb, ng, nf, db = c_int32(), c_int32(), c_int32(), c_size_t()
@@ -170,7 +178,10 @@ class Plan:
         f = np.zeros((self.n_fbuckets, 2), dtype=np.int32)
         _check(lib().shampoo_plan_tables(self.handle, b.ctypes.data_as(P(c_int32)), g.ctypes.data_as(P(c_int32)),
                                          f.ctypes.data_as(P(c_int32))), "shampoo_plan_tables")
-        return {"blocks": b, "g_buckets": g, "f_buckets": f}
+        sides = np.zeros(self.n_fbuckets, dtype=np.int32)
+        _check(lib().shampoo_plan_factor_sides(self.handle, sides.ctypes.data_as(P(c_int32))),
+               "shampoo_plan_factor_sides")
+        return {"blocks": b, "g_buckets": g, "f_buckets": f, "f_sides": sides}
 
     def bind(self, device="cuda", stream=None):
         import torch

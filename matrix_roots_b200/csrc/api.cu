@@ -21,6 +21,7 @@ struct shp_plan {
   std::vector<int32_t> blocks;      // n_blocks x kBlockFields
   std::vector<int32_t> gb;          // n_gbuckets x 3 (rows, cols, count)
   std::vector<int32_t> fb;          // n_fbuckets x 2 (n, count)
+  std::vector<int32_t> gside, fside;  // per bucket: 0 two-sided, 1 one-sided (left factors only)
   // device table image: blocks | per gbucket (l_idx, r_idx) | layer_first | gstack_off
   std::vector<int32_t> image;
   std::vector<size_t> off_lidx, off_ridx;
@@ -564,11 +565,11 @@ shp_status shampoo_device_error(int32_t* out) {
 
 shp_status shampoo_plan_create(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
                                shp_plan** plan_out) {
-  return shampoo_plan_create_ex(rows, cols, n_layers, block_size, 0, plan_out);
+  return shampoo_plan_create_ex(rows, cols, nullptr, n_layers, block_size, 0, plan_out);
 }
 
-shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int32_t n_layers, int32_t block_size,
-                                  int32_t flags, shp_plan** plan_out) {
+shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, const int32_t* left_only,
+                                  int32_t n_layers, int32_t block_size, int32_t flags, shp_plan** plan_out) {
   if (!plan_out) return fail(SHP_ERR_INVALID_ARG, "plan_out is NULL");
   if (flags & ~SHP_PLAN_LAYERWISE) return fail(SHP_ERR_INVALID_ARG, "unknown plan flags 0x%x", flags);
   const bool layerwise = (flags & SHP_PLAN_LAYERWISE) != 0;
@@ -585,15 +586,16 @@ shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int3
   std::vector<int> rs, cs;
   std::vector<int> fkey, flayer;  // factor bucket n values (and layers, when layerwise) in order
   std::vector<int> glayer;        // gradient bucket layers, when layerwise
-  int cur_layer = 0;
+  int cur_layer = 0, cur_side = 0;
   auto fslot = [&](int n, int32_t* bucket, int32_t* index) {
     int b = -1;
     for (size_t i = 0; i < fkey.size(); ++i)
-      if (fkey[i] == n && (!layerwise || flayer[i] == cur_layer)) b = (int)i;
+      if (fkey[i] == n && p->fside[i] == cur_side && (!layerwise || flayer[i] == cur_layer)) b = (int)i;
     if (b < 0) {
       b = (int)fkey.size();
       fkey.push_back(n);
       flayer.push_back(cur_layer);
+      p->fside.push_back(cur_side);
       p->fb.push_back(n);
       p->fb.push_back(0);
     }
@@ -602,6 +604,7 @@ shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int3
   };
   for (int l = 0; l < n_layers; ++l) {
     cur_layer = l;
+    cur_side = left_only && left_only[l] ? 1 : 0;
     split_dim(rows[l], block_size, rs);
     split_dim(cols[l], block_size, cs);
     const size_t first = p->blocks.size();
@@ -616,10 +619,12 @@ shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int3
         }
         int g = -1;
         for (int i = 0; i < (int)p->gb.size() / 3; ++i)
-          if (p->gb[3 * i] == r && p->gb[3 * i + 1] == c && (!layerwise || glayer[i] == l)) g = i;
+          if (p->gb[3 * i] == r && p->gb[3 * i + 1] == c && p->gside[i] == cur_side && (!layerwise || glayer[i] == l))
+            g = i;
         if (g < 0) {
           g = (int)p->gb.size() / 3;
           glayer.push_back(l);
+          p->gside.push_back(cur_side);
           p->gb.push_back(r);
           p->gb.push_back(c);
           p->gb.push_back(0);
@@ -636,7 +641,7 @@ shp_status shampoo_plan_create_ex(const int32_t* rows, const int32_t* cols, int3
       int32_t* rec = &p->blocks[first + i * kBlockFields];
       fslot(rec[5], &rec[9], &rec[10]);
     }
-    for (size_t i = 0; i < nb; ++i) {  // then its right factors
+    for (size_t i = 0; i < nb && !cur_side; ++i) {  // then its right factors (two-sided layers)
       int32_t* rec = &p->blocks[first + i * kBlockFields];
       fslot(rec[6], &rec[11], &rec[12]);
     }
@@ -699,6 +704,12 @@ shp_status shampoo_plan_tables(const shp_plan* plan, int32_t* blocks, int32_t* g
   if (blocks) memcpy(blocks, plan->blocks.data(), plan->blocks.size() * sizeof(int32_t));
   if (gbuckets) memcpy(gbuckets, plan->gb.data(), plan->gb.size() * sizeof(int32_t));
   if (fbuckets) memcpy(fbuckets, plan->fb.data(), plan->fb.size() * sizeof(int32_t));
+  return SHP_OK;
+}
+
+shp_status shampoo_plan_factor_sides(const shp_plan* plan, int32_t* sides) {
+  if (!plan || !sides) return fail(SHP_ERR_INVALID_ARG, "plan and sides must be non-NULL");
+  memcpy(sides, plan->fside.data(), plan->fside.size() * sizeof(int32_t));
   return SHP_OK;
 }
 
@@ -806,6 +817,7 @@ shp_status shampoo_update_stats(const shp_plan* plan, const float* const* g_stac
     gs[1].epi.o_idx = plan->dev + plan->off_ridx[g];
     gs[1].epi.alpha = alpha;
     gs[1].epi.beta = beta2;
+    if (rb < 0) rb = lb;  // one-sided bucket: the second problem is not launched
     gs[1].epi.C.f32 = f_stacks[rb];
     gs[1].epi.C.ld = n;
     gs[1].epi.C.bs = (long long)n * n;
@@ -814,7 +826,8 @@ shp_status shampoo_update_stats(const shp_plan* plan, const float* const* g_stac
       gs[0].epi.C = EpiC();
       gs[1].epi.C = EpiC();
     }
-    cudaError_t e = launch_gemm(gs, 2, cnt, pr, st);
+    const int nprob = plan->gside[g] ? 1 : 2;  // one-sided: no right factor
+    cudaError_t e = launch_gemm(gs, nprob, cnt, pr, st);
     if (e != cudaSuccess) return fail(SHP_ERR_CUDA, "statistics GEMM: %s", cudaGetErrorString(e));
   }
   return SHP_OK;
@@ -968,7 +981,8 @@ shp_status shampoo_precondition(const shp_plan* plan, const float* const* roots,
         break;
       }
     }
-    if (!roots[lb] || !roots[rb] || !g_stacks[g] || !d_stacks[g])
+    const bool one_sided = plan->gside[g] != 0;
+    if (!roots[lb] || (!one_sided && !roots[rb]) || !g_stacks[g] || !d_stacks[g])
       return fail(SHP_ERR_INVALID_ARG, "NULL stack pointer for gradient bucket %d", g);
     Carver c(workspace);
     PrecBufs b = carve_prec(c, cnt, m, n, pr);
@@ -976,6 +990,14 @@ shp_status shampoo_precondition(const shp_plan* plan, const float* const* roots,
                               st));
     CUDA_TRY(launch_to_planes(roots[lb], m, (long long)m * m, plan->dev + plan->off_lidx[g], cnt, m, m, 1.f, 0.f, 0.f,
                               nullptr, b.XL, pr, st));
+    if (one_sided) {  // D = X_L G
+      GemmGroup g1 = group(m, n, m, &b.XL, 0, &b.G, 1);
+      g1.epi.O = plain_out(d_stacks[g], n, (long long)m * n);
+      g1.epi.sumsq = block_dnorm2 + gstack[g];
+      cudaError_t e = launch_gemm(&g1, 1, cnt, pr, st);
+      if (e != cudaSuccess) return fail(SHP_ERR_CUDA, "precondition GEMM: %s", cudaGetErrorString(e));
+      continue;
+    }
     CUDA_TRY(launch_to_planes(roots[rb], n, (long long)n * n, plan->dev + plan->off_ridx[g], cnt, n, n, 1.f, 0.f, 0.f,
                               nullptr, b.XR, pr, st));
     GemmGroup g1 = group(m, n, n, &b.G, 0, &b.XR, 1);  // P = G X_R

@@ -5,7 +5,12 @@ With ``precond_every`` = f > 1 the roots are recomputed only on steps 1,
 optimizer" README, Hyperparameters: preconditioning_compute_steps; DASH §1,
 roots every 10-100 steps); the statistics are updated every step.
 Method "evd" takes the roots from shampoo_inv_root_evd (blocks up to 128)
-with the dampening heuristic ``evd_heuristic`` (DASH B.1-B.2).
+with the dampening heuristic ``evd_heuristic`` (DASH B.1-B.2).  Layers
+listed in ``one_sided`` keep only left statistics and step along
+L^(-1/2) G ("Shampoo" notes, "Roots on idle CPUs": embeddings, softmax and
+layers too large for a right factor).  ``matrix_view`` gives the matrix an
+N-d parameter is preconditioned as (DASH D: a (E, 3, 16, 16) patch
+embedding becomes (E, 768)).
 
 ``BlockedShampoo`` owns the device state (gradient / factor / root /
 direction stacks, graft moments and one shared workspace) and calls, in
@@ -20,6 +25,25 @@ from dataclasses import dataclass
 
 from . import binding as B
 from . import workloads
+
+
+def matrix_shape(shape):
+    """(first dimension, product of the rest) for rank >= 2; None for rank
+    0 and 1 (left to a diagonal optimizer)."""
+    shape = tuple(int(x) for x in shape)
+    if len(shape) < 2:
+        return None
+    rest = 1
+    for x in shape[1:]:
+        rest *= x
+    return (shape[0], rest)
+
+
+def matrix_view(t):
+    """The 2-D view of a contiguous parameter or gradient tensor that the
+    optimizer preconditions (``matrix_shape``); None for vectors."""
+    shp = matrix_shape(t.shape)
+    return None if shp is None else t.view(shp)
 
 
 @dataclass
@@ -49,6 +73,7 @@ class ShampooConfig:
     graph: bool = False         # replay the launches before the graft step as a CUDA graph
     layerwise: bool = False     # stack per layer instead of across all layers
     evd_heuristic: str = "corrected"  # method "evd": corrected, shifted_relu, abs_add or shmp
+    one_sided: tuple = ()       # layer indices preconditioned on the left only, D = L^(-1/2) G
 
 
 class BlockedShampoo:
@@ -57,7 +82,8 @@ class BlockedShampoo:
         self.cfg = cfg
         self.device = torch.device(device)
         self.shapes = [(int(m), int(n)) for m, n in shapes]
-        self.plan = B.Plan(self.shapes, cfg.block_size, cfg.layerwise).bind(self.device)
+        left_only = [i in set(cfg.one_sided) for i in range(len(self.shapes))] if cfg.one_sided else None
+        self.plan = B.Plan(self.shapes, cfg.block_size, cfg.layerwise, left_only).bind(self.device)
         t = self.plan.tables()
         self.tables = t
         f32 = dict(dtype=torch.float32, device=self.device)
@@ -93,11 +119,12 @@ class BlockedShampoo:
         B.stack_blocks(self.plan, G, self.g_stacks, stream)
         B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
         for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
+            p = 2 if self.tables["f_sides"][fb] else c.root_p  # one-sided layers: L^(-1/2)
             if c.method == "evd":
-                B.inv_root_evd(self.factors[fb], c.eps, c.evd_heuristic, c.root_p, out=self.roots[fb],
+                B.inv_root_evd(self.factors[fb], c.eps, c.evd_heuristic, p, out=self.roots[fb],
                                status_out=self.status[fb], stream=stream)
                 continue
-            B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, c.root_p, c.pi_vectors, c.pi_iters,
+            B.inv_root(self.factors[fb], c.eps, c.method, c.iters, c.dtype, c.scaling, p, c.pi_vectors, c.pi_iters,
                        self.pi_starts.get(int(n)), self.roots[fb], self.scales[fb], self.status[fb], ws, stream)
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,
                        stream)

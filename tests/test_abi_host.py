@@ -61,7 +61,7 @@ def test_plan_tables_bit_exact_with_oracle(shapes, bs, layerwise):
     plan = B.Plan(shapes, bs, layerwise)
     got = plan.tables()
     ref = O.plan_blocks(shapes, bs, layerwise)
-    for k in ("blocks", "g_buckets", "f_buckets"):
+    for k in ("blocks", "g_buckets", "f_buckets", "f_sides"):
         assert got[k].dtype == np.int32
         assert np.array_equal(got[k], ref[k]), k
 
@@ -74,10 +74,22 @@ def test_plan_random_shapes_bit_exact():
         if bs == 0:
             shapes = [(min(m, 4096), min(n, 4096)) for m, n in shapes]
         lw = bool(rng.integers(0, 2))
-        got = B.Plan(shapes, bs, lw).tables()
-        ref = O.plan_blocks(shapes, bs, lw)
-        for k in ("blocks", "g_buckets", "f_buckets"):
-            assert np.array_equal(got[k], ref[k]), (shapes, bs, lw, k)
+        lo = [bool(x) for x in rng.integers(0, 2, len(shapes))] if rng.integers(0, 2) else None
+        got = B.Plan(shapes, bs, lw, lo).tables()
+        ref = O.plan_blocks(shapes, bs, lw, lo)
+        for k in ("blocks", "g_buckets", "f_buckets", "f_sides"):
+            assert np.array_equal(got[k], ref[k]), (shapes, bs, lw, lo, k)
+
+
+@pytest.mark.parametrize("layerwise", [False, True])
+def test_plan_one_sided_bit_exact_with_oracle(layerwise):
+    shapes = W.transformer_shapes()[:6] + [(200, 136), (64, 300)]
+    lo = [i % 3 == 1 for i in range(len(shapes))]
+    got = B.Plan(shapes, 512, layerwise, lo).tables()
+    ref = O.plan_blocks(shapes, 512, layerwise, lo)
+    for k in ("blocks", "g_buckets", "f_buckets", "f_sides"):
+        assert np.array_equal(got[k], ref[k]), k
+    assert got["f_sides"].sum() > 0
 
 
 def test_plan_unknown_flags_refused():
@@ -85,7 +97,7 @@ def test_plan_unknown_flags_refused():
     rows = (ctypes.c_int32 * 1)(64)
     cols = (ctypes.c_int32 * 1)(64)
     h = ctypes.c_void_p()
-    assert L.shampoo_plan_create_ex(rows, cols, 1, 64, 2, ctypes.byref(h)) == B.SHP_ERR_INVALID_ARG
+    assert L.shampoo_plan_create_ex(rows, cols, None, 1, 64, 2, ctypes.byref(h)) == B.SHP_ERR_INVALID_ARG
 
 
 def test_plan_rejects_bad_input():

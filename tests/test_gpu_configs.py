@@ -165,6 +165,39 @@ def test_inv_root_warm_matches_oracle(n, p):
         assert rel(X[b], ref) < 1e-3, (b, rel(X[b], ref))
 
 
+def test_one_sided_layers_in_the_step():
+    """A model with one one-sided layer (D = L^(-1/2) G) among two-sided
+    ones, and an N-d parameter taken through its matrix view: 3 steps,
+    Newton-DB-20 FP32 (one call for the square roots), damping 1 so every
+    factor is well conditioned, Adam graft; the stated 1e-3 on W against the
+    oracle's step with the same one-sided layer."""
+    import torch
+    from matrix_roots_b200.optimizer import matrix_view
+    shapes = [(128, 256), (96, 64), (64, 3, 8, 8)]
+    mats = [tuple(O.matrix_shape(s)) for s in shapes]
+    assert mats[2] == (64, 192)
+    rng = np.random.default_rng(13)
+    G = [[rng.standard_normal(s).astype(np.float32) for s in shapes] for _ in range(3)]
+    cfg = ShampooConfig(block_size=64, beta2=0.999, alpha=1.0, eps=1.0, method="ndb", iters=20, dtype="fp32",
+                        scaling="frobenius", graft="adam", lr=1e-2, one_sided=(1,))
+    opt = BlockedShampoo(mats, cfg)
+    assert int(opt.tables["f_sides"].sum()) > 0
+    Wt = [torch.zeros(s, device="cuda") for s in shapes]
+    st = O.ShampooState(mats, 64, "adam", left_only=[False, True, False])
+    Wr = [np.zeros(m) for m in mats]
+    for t in range(3):
+        Gt = [to_dev(g) for g in G[t]]
+        opt.step([matrix_view(w) for w in Wt], [matrix_view(g) for g in Gt])
+        Wr = O.shampoo_step(st, Wr, [g.reshape(m).astype(np.float64) for g, m in zip(G[t], mats)], beta2=0.999,
+                            alpha=1.0, eps=1.0, method="ndb", iters=20, scaling="frobenius", graft="adam", lr=1e-2)
+        torch.cuda.synchronize()
+        for li in range(len(shapes)):
+            err = rel(Wt[li].cpu().numpy().reshape(mats[li]), Wr[li])
+            print(f"one-sided model step {t + 1}, layer {li}: {err:.2e}")
+            assert err < 1e-3
+    assert all((s.cpu().numpy() == 0).all() for s in opt.status)
+
+
 def test_stale_roots_every_third_step():
     """Preconditioner frequency f = 3 on the tiny dense workload (6 steps,
     NDB-20 FP32): statistics every step, roots on steps 1 and 4 only.  As for

@@ -9,10 +9,11 @@
 // n + 1, so row and column sweeps are both free of bank conflicts; that
 // bounds n at 128 (128 x 129 x (8 + 4) B = 198 KB).  The eigensolver is
 // two-sided cyclic Jacobi in the round-robin pair order: each round rotates
-// n/2 disjoint (p, q) planes at once, one warp per plane: the warp works
-// out its plane's rotation and rotates the two rows, and after a barrier the
-// same warps rotate the two columns of A and of V (two barriers a round).
-// A plane is
+// n/2 disjoint (p, q) planes at once.  The rotations are worked out first;
+// after a barrier, A <- J^T A J is applied one 2 x 2 block (two rows of one
+// plane, two columns of another) at a time in registers, V <- V J alongside,
+// so every entry of A and V is read and written once a round (two barriers
+// a round).  A plane is
 // rotated only while its off-diagonal entry is above 2^-21 sqrt(|a_pp
 // a_qq|); a sweep without rotations ends the solve.  Then X = V diag(f(mu))
 // V^T with f the chosen heuristic, written row-major in float32.
@@ -57,7 +58,7 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
     evd_root_kernel(const float* __restrict__ A, int n, float eps, int p, int heuristic, float* __restrict__ X,
                     float* __restrict__ eig, int* __restrict__ status) {
   extern __shared__ double smem[];
-  __shared__ int pr_p[64], pr_q[64];
+  __shared__ int pr_x[64], pr_y[64];
   __shared__ double pr_s[64], pr_tau[64], pr_t[64], pr_app[64], pr_aqq[64], pr_apq[64];
   __shared__ float fval[128];
   __shared__ int rotated, flags;
@@ -99,79 +100,99 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
   int sweeps = 0;
   for (; sweeps < kEvdMaxSweeps && !converged; ++sweeps) {
     for (int round = 0; round < m - 1; ++round) {
-      // Rotation angles and rows: warp w owns pairs w, w + 16, ...; its
-      // lanes read the pivot entries (broadcast), agree on the rotation,
-      // then rotate rows p and q, 32 columns at a time.  No other warp
-      // touches those two rows in this phase.
-      for (int k = warp; k < half; k += kEvdWarps) {
-        int P = k == 0 ? 0 : 1 + (k - 1 + round) % (m - 1);
-        int Q = 1 + (m - 2 - k + round) % (m - 1);
-        if (P > Q) {
-          const int t = P;
-          P = Q;
-          Q = t;
-        }
-        double s = 0.0, tau2 = 0.0, t = 0.0, app = 0.0, aqq = 0.0, apq = 0.0;
-        if (Q < n) {
-          app = a[P * ld + P];
-          aqq = a[Q * ld + Q];
-          apq = a[P * ld + Q];
-          if (apq != 0.0 && fabs(apq) > kRelTol * sqrt(fabs(app) * fabs(aqq))) {
-            // tan of the angle that zeroes a_pq, the smaller root (|t| <= 1)
-            const double th = (aqq - app) / (2.0 * apq);
+      // Rotations of this round's planes (X, Y) = (players at positions k
+      // and m-1-k; the formulas need no ordering).
+      for (int k = tid; k < half; k += blockDim.x) {
+        const int X = k == 0 ? 0 : 1 + (k - 1 + round) % (m - 1);
+        const int Y = 1 + (m - 2 - k + round) % (m - 1);
+        double s = 0.0, tau2 = 0.0, t = 0.0, axx = 0.0, ayy = 0.0, axy = 0.0;
+        if (X < n && Y < n) {
+          axx = a[X * ld + X];
+          ayy = a[Y * ld + Y];
+          axy = a[X * ld + Y];
+          if (axy != 0.0 && fabs(axy) > kRelTol * sqrt(fabs(axx) * fabs(ayy))) {
+            // tan of the angle that zeroes a_xy, the smaller root (|t| <= 1)
+            const double th = (ayy - axx) / (2.0 * axy);
             const double ath = fabs(th);
             t = ath > 1e150 ? 0.5 / th : copysign(1.0, th) / (ath + sqrt(1.0 + th * th));
             const double c = 1.0 / sqrt(1.0 + t * t);
             s = t * c;
             tau2 = s / (1.0 + c);
+            rotated = 1;
           }
         }
-        if (lane == 0) {
-          pr_p[k] = P;
-          pr_q[k] = Q;
-          pr_s[k] = s;
-          pr_tau[k] = tau2;
-          pr_t[k] = t;
-          pr_app[k] = app;
-          pr_aqq[k] = aqq;
-          pr_apq[k] = apq;
-          if (s != 0.0) rotated = 1;
-        }
-        __syncwarp();  // every lane has read the pivot entries
-        if (s == 0.0) continue;
-        double* rp = a + P * ld;
-        double* rq = a + Q * ld;
-        for (int j = lane; j < n; j += 32) {
-          const double x = rp[j], y = rq[j];
-          rp[j] = x - s * (y + tau2 * x);
-          rq[j] = y + s * (x - tau2 * y);
-        }
+        pr_x[k] = X;
+        pr_y[k] = Y;
+        pr_s[k] = s;
+        pr_tau[k] = tau2;
+        pr_t[k] = t;
+        pr_app[k] = axx;
+        pr_aqq[k] = ayy;
+        pr_apq[k] = axy;
       }
       __syncthreads();
-      // columns p, q of A and V <- . J; the 2 x 2 pivot block set exactly
+      // A <- J^T A J and V <- V J one 2 x 2 block at a time: block (k, kc)
+      // holds rows X_k, Y_k and columns X_kc, Y_kc; it is rotated by plane
+      // k on the left and plane kc on the right, in registers.  Warp w takes
+      // row planes w, w + 16, ...; its lanes take consecutive column planes,
+      // whose columns are consecutive players (conflict-free).
       for (int k = warp; k < half; k += kEvdWarps) {
-        const double s = pr_s[k];
-        if (s == 0.0) continue;
-        const double tau2 = pr_tau[k];
-        const int P = pr_p[k], Q = pr_q[k];
-        const float sf = (float)s, tf = (float)tau2;
-        for (int r = lane; r < n; r += 32) {
-          double* ar = a + r * ld;
-          const double x = ar[P], y = ar[Q];
-          double nx = x - s * (y + tau2 * x), ny = y + s * (x - tau2 * y);
-          if (r == P) {
-            nx = pr_app[k] - pr_t[k] * pr_apq[k];
-            ny = 0.0;
-          } else if (r == Q) {
-            nx = 0.0;
-            ny = pr_aqq[k] + pr_t[k] * pr_apq[k];
+        const int X = pr_x[k], Y = pr_y[k];
+        const bool xv = X < n, yv = Y < n;
+        const double s = pr_s[k], tau2 = pr_tau[k];
+        for (int kc = lane; kc < half; kc += 32) {
+          const double sc = pr_s[kc];
+          if (s == 0.0 && sc == 0.0) continue;
+          const double tc = pr_tau[kc];
+          const int Xc = pr_x[kc], Yc = pr_y[kc];
+          const bool xcv = Xc < n, ycv = Yc < n;
+          double* ax = a + X * ld;
+          double* ay = a + Y * ld;
+          double b00 = (xv && xcv) ? ax[Xc] : 0.0, b01 = (xv && ycv) ? ax[Yc] : 0.0;
+          double b10 = (yv && xcv) ? ay[Xc] : 0.0, b11 = (yv && ycv) ? ay[Yc] : 0.0;
+          if (s != 0.0) {  // rows X, Y <- J_k^T
+            double u = b00, w = b10;
+            b00 = u - s * (w + tau2 * u);
+            b10 = w + s * (u - tau2 * w);
+            u = b01;
+            w = b11;
+            b01 = u - s * (w + tau2 * u);
+            b11 = w + s * (u - tau2 * w);
           }
-          ar[P] = nx;
-          ar[Q] = ny;
-          float* vr = v + r * ld;
-          const float vx = vr[P], vy = vr[Q];
-          vr[P] = vx - sf * (vy + tf * vx);
-          vr[Q] = vy + sf * (vx - tf * vy);
+          if (sc != 0.0) {  // columns X_kc, Y_kc <- . J_kc
+            double u = b00, w = b01;
+            b00 = u - sc * (w + tc * u);
+            b01 = w + sc * (u - tc * w);
+            u = b10;
+            w = b11;
+            b10 = u - sc * (w + tc * u);
+            b11 = w + sc * (u - tc * w);
+          }
+          if (kc == k && s != 0.0) {  // the pivot block, exactly
+            b00 = pr_app[k] - pr_t[k] * pr_apq[k];
+            b11 = pr_aqq[k] + pr_t[k] * pr_apq[k];
+            b01 = 0.0;
+            b10 = 0.0;
+          }
+          if (xv && xcv) ax[Xc] = b00;
+          if (xv && ycv) ax[Yc] = b01;
+          if (yv && xcv) ay[Xc] = b10;
+          if (yv && ycv) ay[Yc] = b11;
+          if (sc != 0.0) {  // V rows X, Y, columns X_kc, Y_kc <- . J_kc
+            const float sf = (float)sc, tf = (float)tc;
+            if (xv) {
+              float* vx = v + X * ld;
+              const float u = vx[Xc], w = vx[Yc];
+              vx[Xc] = u - sf * (w + tf * u);
+              vx[Yc] = w + sf * (u - tf * w);
+            }
+            if (yv) {
+              float* vy = v + Y * ld;
+              const float u = vy[Xc], w = vy[Yc];
+              vy[Xc] = u - sf * (w + tf * u);
+              vy[Yc] = w + sf * (u - tf * w);
+            }
+          }
         }
       }
       __syncthreads();

@@ -72,18 +72,23 @@ def make_grads(shapes, seed, kind="transformer"):
     return W.transformer_grads(shapes, seed=seed)
 
 
-GEMM_DRAM_BYTES_PER_LAUNCH = 3744.1e6
+# DRAM bytes per launch of the FP32 GEMM on the transformer workload, from
+# the ncu launch list of the current kernel; None until it is captured
+GEMM_DRAM_BYTES_PER_LAUNCH = None
 
 
-def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters):
-    """Algorithmic FLOPs of one shampoo_inv_root call (2 n^3 per matmul)."""
+def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters, dense=False):
+    """Algorithmic FLOPs of one shampoo_inv_root call: 2 n^3 per product of
+    the coupled iterations; the Chebyshev products are computed as symmetric
+    matrices, so their algorithmic work is that of the n(n+1)/2 distinct
+    entries, n^2 (n+1) flops (``dense`` counts 2 n^3 for them too)."""
     if method == "ndb":
         mm = 2 * (3 * iters - 3) if iters >= 2 else 2
     elif method == "cn":
         mm = 4 * iters - 4 if iters >= 2 else 0
     else:
         mm = max(iters - 1, 0)
-    f = mm * 2.0 * n ** 3
+    f = mm * (n * n * (n + 1.0) if (method == "cheb" and not dense) else 2.0 * n ** 3)
     if scaling == "power":
         f += (pi_iters + 1) * 2.0 * n * n * pi_vectors
     return f * count
@@ -409,9 +414,8 @@ def run_ours(args, cfg):
     passes = {"fp32": 3.0, "tf32": 2.0, "fp16": 1.0, "bf16": 1.0}[args.dtype]
     peak = peaks["bf16_sust"] / passes
     achieved = flops / (root_ms / 1000.0) / 1e12
-    # DRAM bytes per launch of the FP32 GEMM on this workload, from the ncu
-    # launch list in profiles/launches_transformer_step.txt (mean over the
-    # 121 captured launches); other workloads / dtypes were not captured
+    # DRAM bytes per launch of the FP32 GEMM on this workload (ncu launch
+    # list of the transformer step); other workloads / dtypes not captured
     traffic = GEMM_DRAM_BYTES_PER_LAUNCH if (args.config == "transformer" and args.dtype == "fp32") else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic, "traffic_unit": "DRAM bytes per launch (read + write)",

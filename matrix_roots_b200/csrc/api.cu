@@ -129,8 +129,17 @@ EpiOut plain_out(float* p, int ld, long long bs) {
   return o;
 }
 
-GemmGroup group(int M, int N, int K, const Planes* A, int a_mn, const Planes* B, int b_mn) {
+// sym = 1: the product is symmetric in exact arithmetic (both operands are
+// polynomials in one symmetric matrix, or G G^T / G^T G, and C is
+// symmetric), so only the tiles on and above the diagonal are computed.
+// Used for the statistics and the Chebyshev recurrence only: mirroring the
+// products of the coupled iterations (Newton-DB: Y T, T Z, Z Y; coupled
+// Newton: X T, T^2, T^p M) breaks the error coupling that keeps them
+// stable -- Newton-DB-20 on 1024^2 factors with kappa ~ 5e6 overflowed on
+// the GPU and in a float32 model, coupled Newton lost a factor 6.
+GemmGroup group(int M, int N, int K, const Planes* A, int a_mn, const Planes* B, int b_mn, int sym = 0) {
   GemmGroup g;
+  g.sym = sym;
   g.M = M;
   g.N = N;
   g.K = K;
@@ -493,7 +502,7 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
   for (int k = degree - 2; k >= 1; --k) {
     // B_k = c_k I + 2 S B_{k+1} - B_{k+2}; three buffers, so that no launch
     // writes a matrix it reads
-    GemmGroup g = group(n, n, n, &S, 0, Bk1, 1);
+    GemmGroup g = group(n, n, n, &S, 0, Bk1, 1, 1);
     g.epi.alpha = 2.f;
     g.epi.beta = -1.f;
     g.epi.gamma = (float)c[k];
@@ -506,7 +515,7 @@ shp_status run_cheb(const float* A, int count, int n, float eps, int degree, int
     Bk = t;
   }
   // result = c_0 I + S B_1 - B_2, times s^(-1/4)
-  GemmGroup g = group(n, n, n, &S, 0, Bk1, 1);
+  GemmGroup g = group(n, n, n, &S, 0, Bk1, 1, 1);
   g.epi.alpha = 1.f;
   g.epi.beta = -1.f;
   g.epi.gamma = (float)c[0];
@@ -804,7 +813,7 @@ shp_status shampoo_update_stats(const shp_plan* plan, const float* const* g_stac
       }
     }
     GemmGroup gs[2];
-    gs[0] = group(m, m, n, &P, 0, &P, 0);  // G G^T
+    gs[0] = group(m, m, n, &P, 0, &P, 0, 1);  // G G^T
     gs[0].a_idx = nullptr;
     gs[0].epi.o_idx = plan->dev + plan->off_lidx[g];
     gs[0].epi.alpha = alpha;
@@ -813,7 +822,7 @@ shp_status shampoo_update_stats(const shp_plan* plan, const float* const* g_stac
     gs[0].epi.C.ld = m;
     gs[0].epi.C.bs = (long long)m * m;
     gs[0].epi.O = plain_out(f_stacks[lb], m, (long long)m * m);
-    gs[1] = group(n, n, m, &P, 1, &P, 1);  // G^T G
+    gs[1] = group(n, n, m, &P, 1, &P, 1, 1);  // G^T G
     gs[1].epi.o_idx = plan->dev + plan->off_ridx[g];
     gs[1].epi.alpha = alpha;
     gs[1].epi.beta = beta2;

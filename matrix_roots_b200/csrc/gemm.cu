@@ -118,13 +118,27 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int t, int BN, 
   Tile x;
   x.grp = t >= p.tiles0 ? 1 : 0;
   int r = x.grp ? t - p.tiles0 : t;
+  x.nk = (p.g[x.grp].K + BKE - 1) / BKE;
+  if (p.g[x.grp].sym) {  // upper triangle of square tiles, row by row
+    const int mt = p.mt[x.grp];
+    const int per = mt * (mt + 1) / 2;
+    x.b = r / per;
+    r -= x.b * per;
+    int mi = 0;
+    while (r >= mt - mi) {
+      r -= mt - mi;
+      ++mi;
+    }
+    x.m0 = mi * 128;
+    x.n0 = (mi + r) * 128;
+    return x;
+  }
   const int per = p.mt[x.grp] * p.nt[x.grp];
   x.b = r / per;
   r -= x.b * per;
   const int mi = r / p.nt[x.grp];
   x.m0 = mi * 128;
   x.n0 = (r - mi * p.nt[x.grp]) * BN;
-  x.nk = (p.g[x.grp].K + BKE - 1) / BKE;
   return x;
 }
 
@@ -312,7 +326,10 @@ __device__ __forceinline__ void put4(const OutPtrs& o, long long off, float4 v) 
 
 __device__ __forceinline__ float max4(float4 v) { return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))); }
 
-template <bool NEED_C, bool HAS_X>
+// TRANS: write the transpose of the staged block at (row0, col0), the
+// mirror image of an off-diagonal tile of a symmetric product; output
+// element (r, c) is then staged element (c, r).
+template <bool NEED_C, bool HAS_X, bool TRANS = false>
 __device__ __forceinline__ void epilogue_block4(const GroupDev& g, const EpiCtx& x, int row0, int col0,
                                                 const float4* stage, int lane, float& ss, int& bad, float& mo,
                                                 float& mx) {
@@ -328,7 +345,19 @@ __device__ __forceinline__ void epilogue_block4(const GroupDev& g, const EpiCtx&
   for (int it = 0; it < 8; ++it) {
     const int r = it * 4 + (lane >> 3);
     if (r >= rmax) continue;
-    const float4 a = stage[r * 8 + (cq ^ (r & 7))];
+    float4 a;
+    if (TRANS) {
+      const float* sf = reinterpret_cast<const float*>(stage);
+      float t4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int sr = 4 * cq + i;  // staged row = output column
+        t4[i] = sf[(sr * 8 + ((r >> 2) ^ (sr & 7))) * 4 + (r & 3)];
+      }
+      a = make_float4(t4[0], t4[1], t4[2], t4[3]);
+    } else {
+      a = stage[r * 8 + (cq ^ (r & 7))];
+    }
     float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
     if (NEED_C) c = *reinterpret_cast<const float4*>(cf + r * cld);
     const int e = row0 + r - col;  // component on the diagonal, if 0..3
@@ -688,6 +717,19 @@ __global__ void __launch_bounds__(448, 1) gemm_kernel(const __grid_constant__ Ge
             else
               epilogue_block4<false, false>(g, ec, r0, c0, stage4, lane, ss, bad, mo, mx);
           }
+          if (g.sym && x.m0 != x.n0) {  // the mirrored block of an off-diagonal tile
+            if (ec.need_c) {
+              if (ec.has_x)
+                epilogue_block4<true, true, true>(g, ec, c0, r0, stage4, lane, ss, bad, mo, mx);
+              else
+                epilogue_block4<true, false, true>(g, ec, c0, r0, stage4, lane, ss, bad, mo, mx);
+            } else {
+              if (ec.has_x)
+                epilogue_block4<false, true, true>(g, ec, c0, r0, stage4, lane, ss, bad, mo, mx);
+              else
+                epilogue_block4<false, false, true>(g, ec, c0, r0, stage4, lane, ss, bad, mo, mx);
+            }
+          }
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) stage[lane * 32 + (c ^ lane)] = __uint_as_float(r[c]);
@@ -889,7 +931,9 @@ cudaError_t launch_gemm(const GemmGroup* groups, int ngroups, int batch, Prec pr
     }
     prm.mt[i] = (G.M + 127) / 128;
     prm.nt[i] = (G.N + BN - 1) / BN;
-    const long long ti = (long long)batch * prm.mt[i] * prm.nt[i];
+    prm.g[i].sym = (G.sym && G.M == G.N && BN == 128 && prm.g[i].vec4) ? 1 : 0;
+    const long long ti = prm.g[i].sym ? (long long)batch * prm.mt[i] * (prm.mt[i] + 1) / 2
+                                      : (long long)batch * prm.mt[i] * prm.nt[i];
     if (i == 0) prm.tiles0 = (int)ti;
     total += ti;
   }

@@ -76,6 +76,9 @@ struct GroupDev {
   int* status = nullptr;
   int root_p = 4;  // the multiplier is bscale^(-1/root_p)
   int vec4 = 0;  // set by the launcher: N, leading dimensions and bases allow 16-byte row segments
+  // set by the launcher from GemmGroup::sym: only the tiles on and above the
+  // diagonal are computed, each off-diagonal one also written transposed
+  int sym = 0;
 };
 
 struct alignas(64) GemmParams {
@@ -102,6 +105,11 @@ struct GemmGroup {
   const Planes* B = nullptr;
   int b_mn = 0;
   const int* b_idx = nullptr;
+  // 1: the product is symmetric in exact arithmetic (both operands are
+  // polynomials in one symmetric matrix, or G G^T / G^T G) and C, when read,
+  // is symmetric: the launcher computes the upper tiles only and mirrors
+  // them (ignored unless M == N, the tile is square and rows are 16-byte)
+  int sym = 0;
   GroupDev epi;  // epilogue part (M/N/K/majors/idx filled by the launcher)
 };
 

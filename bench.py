@@ -72,9 +72,10 @@ def make_grads(shapes, seed, kind="transformer"):
     return W.transformer_grads(shapes, seed=seed)
 
 
-# DRAM bytes per launch of the FP32 GEMM on the transformer workload, from
-# the ncu launch list of the current kernel; None until it is captured
-GEMM_DRAM_BYTES_PER_LAUNCH = None
+# DRAM bytes per launch of the FP32 GEMM on the transformer workload: mean
+# over the 121 launches of the ncu launch list in
+# profiles/launches_transformer_step.txt (current kernel)
+GEMM_DRAM_BYTES_PER_LAUNCH = 3482.4e6
 
 
 def root_flops(n, count, method, iters, scaling, pi_vectors, pi_iters, dense=False):

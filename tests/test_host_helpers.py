@@ -1,0 +1,41 @@
+"""Host-side helpers that need no GPU: the matrix view of N-d parameters
+(DASH D: a (E, 3, 16, 16) patch embedding is preconditioned as (E, 768)),
+the optimizer's one-sided layer selection and the EVD work count that
+bench.py reports against the FP64 peak."""
+import numpy as np
+import pytest
+
+import oracle as O
+from matrix_roots_b200 import optimizer as OPT
+
+
+@pytest.mark.parametrize("shape", [(384, 3, 16, 16), (512, 5, 5, 64), (7, 9), (10,), (), (4, 1, 1)])
+def test_matrix_shape_matches_the_oracle_reading(shape):
+    assert OPT.matrix_shape(shape) == O.matrix_shape(shape)
+
+
+def test_matrix_view_is_a_view():
+    import torch
+    t = torch.arange(2 * 3 * 4 * 5, dtype=torch.float32).reshape(2, 3, 4, 5)
+    v = OPT.matrix_view(t)
+    assert v.shape == (2, 60) and v.data_ptr() == t.data_ptr()
+    v[1, 7] = -1.0
+    assert t.reshape(-1)[67] == -1.0
+    assert OPT.matrix_view(torch.zeros(5)) is None
+
+
+def test_evd_work_count():
+    import bench
+    # one sweep of a 4 x 4 matrix: 6 rotations, 16 * 4 flops each
+    assert bench.evd_fp64_flops(4, np.array([1])) == 6 * 16 * 4
+    assert bench.evd_fp64_flops(128, np.array([10, 20])) == 30 * (128 * 127 / 2) * 16 * 128
+
+
+def test_root_flop_counts():
+    import bench
+    n = 1024
+    # Newton-DB-20: two calls of 1 + 3 * 19 products; dense products
+    assert bench.root_flops(n, 1, "ndb", 20, "frobenius", 16, 10) == 2 * 57 * 2.0 * n ** 3
+    # Chebyshev products are symmetric: n^2 (n + 1) each, d - 1 of them
+    assert bench.root_flops(n, 2, "cheb", 32, "frobenius", 16, 10) == 2 * 31 * n * n * (n + 1.0)
+    assert bench.root_flops(n, 1, "cheb", 32, "frobenius", 16, 10, dense=True) == 31 * 2.0 * n ** 3

@@ -3,7 +3,9 @@
 With ``precond_every`` = f > 1 the roots are recomputed only on steps 1,
 1 + f, ... and the stale roots precondition the steps between ("3D-Shampoo
 optimizer" README, Hyperparameters: preconditioning_compute_steps; DASH §1,
-roots every 10-100 steps); the statistics are updated every step.
+roots every 10-100 steps); the statistics are updated on steps 1,
+1 + s, ... with ``stats_every`` = s (statistics_compute_steps; default
+every step).
 Method "evd" takes the roots from shampoo_inv_root_evd (blocks up to 128)
 with the dampening heuristic ``evd_heuristic`` (DASH B.1-B.2).  Layers
 listed in ``one_sided`` keep only left statistics and step along
@@ -68,7 +70,8 @@ class ShampooConfig:
     graft_eps: float = 1e-8
     weight_decay: float = 0.0
     graft_per_block: bool = False
-    precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...; statistics every step
+    precond_every: int = 1      # roots on steps 1, 1+f, 1+2f, ...
+    stats_every: int = 1        # statistics on steps 1, 1+s, 1+2s, ...
     root_p: int = 4             # inverse p-th roots, p in (2, 4, 8)
     graph: bool = False         # replay the launches before the graft step as a CUDA graph
     layerwise: bool = False     # stack per layer instead of across all layers
@@ -112,12 +115,14 @@ class BlockedShampoo:
         self._graphs = {}       # (fresh roots?, gradient addresses) -> (CUDAGraph, library launches in it)
         self.graph_launches = 0  # library kernel launches replayed from graphs so far
 
-    def _direction(self, G, stream, fresh: bool) -> None:
-        """Stack, statistics, roots (when fresh) and D for gradients G."""
+    def _direction(self, G, stream, fresh: bool, stats: bool = True) -> None:
+        """Stack, statistics (when ``stats``), roots (when fresh) and D for
+        gradients G."""
         c = self.cfg
         ws = self.workspace
         B.stack_blocks(self.plan, G, self.g_stacks, stream)
-        B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
+        if stats:
+            B.update_stats(self.plan, self.g_stacks, self.factors, c.beta2, c.alpha, c.stats_dtype, ws, stream)
         for fb, (n, _) in enumerate(self.tables["f_buckets"] if fresh else []):
             p = 2 if self.tables["f_sides"][fb] else c.root_p  # one-sided layers: L^(-1/2)
             if c.method == "evd":
@@ -129,23 +134,23 @@ class BlockedShampoo:
         B.precondition(self.plan, self.roots, self.g_stacks, self.d_stacks, self.dnorm2, c.precond_dtype, ws,
                        stream)
 
-    def _direction_graphed(self, G, fresh: bool) -> None:
+    def _direction_graphed(self, G, fresh: bool, stats: bool = True) -> None:
         """The same launches replayed from a CUDA graph captured on the first
         step that sees these gradient tensors (their addresses are part of
         the graph: refill the same tensors every step).  The first such step
         runs eagerly, so every kernel is set up before the capture."""
         import torch
-        key = (fresh, tuple(int(g.data_ptr()) for g in G))
+        key = (fresh, stats, tuple(int(g.data_ptr()) for g in G))
         if key not in self._graphs:
             if (None,) + key not in self._graphs:
                 self._graphs[(None,) + key] = None  # seen once: run eagerly
-                self._direction(G, None, fresh)
+                self._direction(G, None, fresh, stats)
                 return
             graph = torch.cuda.CUDAGraph()
             before = B.launch_count()
             torch.cuda.synchronize(self.device)
             with torch.cuda.graph(graph):
-                self._direction(G, None, fresh)
+                self._direction(G, None, fresh, stats)
             self._graphs[key] = (graph, B.launch_count() - before)
         graph, n = self._graphs[key]
         graph.replay()
@@ -160,9 +165,10 @@ class BlockedShampoo:
         ws = self.workspace
         self.t += 1
         fresh = (self.t - 1) % max(int(c.precond_every), 1) == 0
+        stats = (self.t - 1) % max(int(c.stats_every), 1) == 0
         if c.graph:
-            self._direction_graphed(G, fresh)
+            self._direction_graphed(G, fresh, stats)
         else:
-            self._direction(G, stream, fresh)
+            self._direction(G, stream, fresh, stats)
         B.graft_step(self.plan, W, G, self.d_stacks, self.dnorm2, self.m, self.v, c.graft, c.lr, c.beta1,
                      c.graft_beta2, c.graft_eps, c.weight_decay, self.t, c.graft_per_block, ws, stream)

@@ -48,7 +48,9 @@ R12 Root power p: p in {2, 4, 8} ([Notes] "Spreading the preconditioners":
     call's Y; coupled Newton and Chebyshev take p directly.
 R11 Preconditioner frequency f: statistics every step, roots on steps
     1, 1+f, 1+2f, ... and the last roots reused in between ([3D-Shampoo]
-    Hyperparameters: preconditioning_compute_steps; [DASH] §1).
+    Hyperparameters: preconditioning_compute_steps; [DASH] §1).  The
+    statistics frequency s (statistics_compute_steps) likewise updates the
+    statistics on steps 1, 1+s, ... only; every step is preconditioned.
 R16 One-sided layers ([Notes] "Roots on idle CPUs": embedding and softmax
     layers, and layers too large for a right factor, are preconditioned on
     one side only, L^{-1/2} G, the alpha = 1 split of the Kronecker bound):
@@ -724,7 +726,8 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
                  method: str, iters: int, scaling: str, graft: str, lr: float,
                  beta1: float = 0.9, graft_beta2: float = 0.999, graft_eps: float = 1e-8,
                  wd: float = 0.0, pi_starts=None, pi_iters: int = 10, scales_out=None,
-                 replay: bool = True, prec=None, precond_every: int = 1, evd_heuristic: str = "corrected"):
+                 replay: bool = True, prec=None, precond_every: int = 1, evd_heuristic: str = "corrected",
+                 stats_every: int = 1):
     """One optimizer step over all layers; returns the new weights.
 
     ``scales_out`` (optional dict) receives the per-factor scale used, keyed by
@@ -738,7 +741,8 @@ def shampoo_step(state: ShampooState, W, grads, *, beta2: float, alpha: float, e
     plan = state.plan
     state.step += 1
     g_st = stack_gradients(plan, grads)
-    for b in plan["blocks"]:
+    stats_step = (state.step - 1) % max(int(stats_every), 1) == 0
+    for b in (plan["blocks"] if stats_step else []):
         gb, gi, lb, lix, rb, rix = (int(x) for x in b[7:13])
         if rb < 0:  # one-sided layer: left statistics only (reading R16)
             g = np.asarray(g_st[gb][gi], dtype=np.float64)

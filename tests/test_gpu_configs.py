@@ -198,6 +198,34 @@ def test_one_sided_layers_in_the_step():
     assert all((s.cpu().numpy() == 0).all() for s in opt.status)
 
 
+def test_statistics_every_second_step():
+    """statistics_compute_steps = 2 with roots every step on the tiny dense
+    workload (5 steps): W against the oracle's step with the same schedule
+    and float64 EVD roots, bound 1e-3 plus the exact Newton-DB-vs-EVD gap on
+    the same schedule (as for the tiny dense test)."""
+    import torch
+    G = W.tiny_dense_grads()
+    shapes = [(256, 256)]
+    cfg = ShampooConfig(block_size=64, beta2=1.0, alpha=1.0, eps=1e-6, method="ndb", iters=20, dtype="fp32",
+                        scaling="frobenius", graft="sgd", lr=0.1, stats_every=2)
+    opt = BlockedShampoo(shapes, cfg)
+    Wd = [torch.zeros(256, 256, device="cuda")]
+    st = {k: O.ShampooState(shapes, 64, "sgd") for k in ("evd", "ndb")}
+    Wr = {k: [np.zeros((256, 256))] for k in st}
+    for t in range(5):
+        opt.step(Wd, [to_dev(G[t])])
+        for k in st:
+            Wr[k] = O.shampoo_step(st[k], Wr[k], [G[t]], beta2=1.0, alpha=1.0, eps=1e-6, method=k, iters=20,
+                                   scaling="frobenius", graft="sgd", lr=0.1, stats_every=2)
+        torch.cuda.synchronize()
+        err = rel(Wd[0].cpu().numpy(), Wr["evd"][0])
+        tol = 1e-3 + rel(Wr["ndb"][0], Wr["evd"][0])
+        print(f"statistics every 2nd step, step {t + 1}: GPU vs EVD {err:.2e} (bound {tol:.2e})")
+        assert err < tol
+    for f in range(len(st["ndb"].factors)):
+        assert rel(opt.factors[f].cpu().numpy(), st["ndb"].factors[f]) < 1e-5
+
+
 def test_stale_roots_every_third_step():
     """Preconditioner frequency f = 3 on the tiny dense workload (6 steps,
     NDB-20 FP32): statistics every step, roots on steps 1 and 4 only.  As for

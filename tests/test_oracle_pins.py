@@ -744,3 +744,18 @@ def test_matrix_shape_merges_trailing_dimensions():
     assert O.matrix_shape((512, 5, 5, 64)) == (512, 1600)
     assert O.matrix_shape((7, 9)) == (7, 9)
     assert O.matrix_shape((10,)) is None and O.matrix_shape(()) is None
+
+
+def test_statistics_frequency_updates_on_schedule():
+    """statistics_compute_steps = 2: the statistics after steps 1..4 hold
+    the gradients of steps 1 and 3 only (beta2 = 1: a plain sum)."""
+    rng = np.random.default_rng(41)
+    G = [rng.standard_normal((8, 6)) for _ in range(4)]
+    st = O.ShampooState([(8, 6)], 0, "sgd")
+    W = [np.zeros((8, 6))]
+    for t in range(4):
+        W = O.shampoo_step(st, W, [G[t]], beta2=1.0, alpha=1.0, eps=1e-3, method="evd", iters=0,
+                           scaling="frobenius", graft="sgd", lr=0.1, stats_every=2)
+    lb, li, rb, ri = (int(x) for x in st.plan["blocks"][0][9:13])
+    assert np.allclose(st.factors[lb][li], G[0] @ G[0].T + G[2] @ G[2].T, rtol=1e-12)
+    assert np.allclose(st.factors[rb][ri], G[0].T @ G[0] + G[2].T @ G[2], rtol=1e-12)

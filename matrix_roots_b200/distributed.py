@@ -46,6 +46,17 @@ def assign_layers(shapes: Sequence, block_size: int, world: int) -> list[int]:
     return owner
 
 
+def local_config(cfg, mine: Sequence[int]):
+    """The configuration of the per-rank optimizer over layers ``mine``:
+    per-layer options (the one-sided layer indices) renumbered to the
+    rank's own layer order; everything else unchanged."""
+    import dataclasses
+    one = set(getattr(cfg, "one_sided", ()) or ())
+    if not one or not dataclasses.is_dataclass(cfg):
+        return cfg
+    return dataclasses.replace(cfg, one_sided=tuple(k for k, i in enumerate(mine) if i in one))
+
+
 class DistributedShampoo:
     """One optimizer step over all layers on ``world`` ranks.
 
@@ -69,7 +80,7 @@ class DistributedShampoo:
                        for k in range(self.world)]
         if local_step is None and self.mine:
             from .optimizer import BlockedShampoo
-            opt = BlockedShampoo([self.shapes[i] for i in self.mine], cfg, device)
+            opt = BlockedShampoo([self.shapes[i] for i in self.mine], local_config(cfg, self.mine), device)
             local_step = opt.step
             self.local = opt
         self.local_step = local_step

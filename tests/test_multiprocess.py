@@ -34,6 +34,15 @@ def test_assign_layers_greedy_and_balanced():
         assert max(loads) <= 1.35 * (sum(loads) / world)
 
 
+def test_local_config_renumbers_one_sided_layers():
+    from matrix_roots_b200.optimizer import ShampooConfig
+    cfg = ShampooConfig(block_size=64, one_sided=(1, 4))
+    loc = D.local_config(cfg, [4, 0, 2])
+    assert loc.one_sided == (0,) and loc.block_size == 64 and cfg.one_sided == (1, 4)
+    assert D.local_config(ShampooConfig(), [0, 1]).one_sided == ()
+    assert D.local_config(_HostCfg(), [0]) is not None
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))

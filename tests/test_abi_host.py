@@ -231,3 +231,28 @@ def _call_evd(**over):
 ])
 def test_inv_root_evd_rejects_before_enqueue(over, code):
     assert _call_evd(**over) == code
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as C99 with every
+    warning on, and a C program links against the library's symbols."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "shampoo.h"\n'
+                   'int main(void) {\n'
+                   '  shp_plan* p = 0;\n'
+                   '  int32_t r = 64, c = 32;\n'
+                   '  if (shampoo_plan_create(&r, &c, 1, 0, &p) != SHP_OK) return 1;\n'
+                   '  shampoo_plan_destroy(p);\n'
+                   '  return shampoo_version() > 0 ? 0 : 2;\n'
+                   '}\n')
+    exe = tmp_path / "use"
+    lib_dir = os.path.dirname(B.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", lib_dir, "-l:" + os.path.basename(B.LIB_PATH),
+                    "-Wl,-rpath," + lib_dir], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0

@@ -55,14 +55,19 @@ def test_stack_blocks_bit_exact(shapes, bs):
 
 # ------------------------------------------------------------------ a2 ------
 
+@pytest.mark.parametrize("bs", [128, 0])
 @pytest.mark.parametrize("dtype,tol", [("fp32", 2e-5), ("tf32", 3e-3), ("fp16", 3e-3), ("bf16", 2e-2)])
-def test_update_stats(dtype, tol):
+def test_update_stats(dtype, tol, bs):
+    """Statistics against float64.  Block size 0 keeps the layers whole, so
+    the factors (200, 136, 64, 300) span two or three 128-wide tiles with a
+    ragged last one: the symmetric products are computed on their upper
+    tiles and mirrored, reading the old statistics at the mirrored places."""
     import torch
     shapes = [(200, 136), (64, 300)]
-    plan = B.Plan(shapes, 128).bind()
+    plan = B.Plan(shapes, bs).bind()
     t = plan.tables()
     grads = _grads(shapes, 2)
-    ref_plan = O.plan_blocks(shapes, 128)
+    ref_plan = O.plan_blocks(shapes, bs)
     g_st = O.stack_gradients(ref_plan, grads)
     rng = np.random.default_rng(3)
     f0 = []

@@ -78,10 +78,39 @@ class ShampooConfig:
     evd_heuristic: str = "corrected"  # method "evd": corrected, shifted_relu, abs_add or shmp
     one_sided: tuple = ()       # layer indices preconditioned on the left only, D = L^(-1/2) G
 
+    def check(self, n_layers: int | None = None) -> None:
+        """Raises ValueError for an option the library would refuse or
+        misread; run before any device memory is allocated."""
+        def one_of(name, value, allowed):
+            if value not in allowed:
+                raise ValueError(f"{name} must be one of {sorted(allowed)}, not {value!r}")
+        one_of("method", self.method, set(B.METHODS) | {"evd"})
+        for name in ("dtype", "stats_dtype", "precond_dtype"):
+            one_of(name, getattr(self, name), set(B.DTYPES))
+        one_of("scaling", self.scaling, set(B.SCALINGS))
+        one_of("graft", self.graft, set(B.GRAFTS))
+        one_of("evd_heuristic", self.evd_heuristic, set(B.EVD_HEURISTICS))
+        one_of("root_p", self.root_p, {2, 4, 8})
+        if self.block_size < 0:
+            raise ValueError("block_size must be >= 0 (0: no blocking)")
+        if self.precond_every < 1 or self.stats_every < 1:
+            raise ValueError("precond_every and stats_every must be >= 1")
+        if self.method != "evd" and not (1 <= self.iters <= 1000 or (self.method == "cheb" and self.iters == 0)):
+            raise ValueError("iters must be in [1, 1000] (a Chebyshev degree may be 0)")
+        if not (self.eps >= 0.0) or self.eps == float("inf"):
+            raise ValueError("eps must be finite and >= 0")
+        if self.scaling == "power" and (self.pi_vectors < 8 or self.pi_vectors > 256 or self.pi_vectors % 8):
+            raise ValueError("pi_vectors must be a multiple of 8 in [8, 256]")
+        if self.method == "evd" and 0 < self.block_size and self.block_size > B.EVD_MAX_N:
+            raise ValueError(f"method 'evd' needs blocks of at most {B.EVD_MAX_N} (block_size {self.block_size})")
+        if n_layers is not None and any(not 0 <= i < n_layers for i in self.one_sided):
+            raise ValueError(f"one_sided indices must name layers 0..{n_layers - 1}")
+
 
 class BlockedShampoo:
     def __init__(self, shapes, cfg: ShampooConfig, device="cuda"):
         import torch
+        cfg.check(len(shapes))
         self.cfg = cfg
         self.device = torch.device(device)
         self.shapes = [(int(m), int(n)) for m, n in shapes]

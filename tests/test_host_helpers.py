@@ -39,3 +39,22 @@ def test_root_flop_counts():
     # Chebyshev products are symmetric: n^2 (n + 1) each, d - 1 of them
     assert bench.root_flops(n, 2, "cheb", 32, "frobenius", 16, 10) == 2 * 31 * n * n * (n + 1.0)
     assert bench.root_flops(n, 1, "cheb", 32, "frobenius", 16, 10, dense=True) == 31 * 2.0 * n ** 3
+
+
+@pytest.mark.parametrize("bad", [
+    dict(method="svd"), dict(dtype="fp64"), dict(scaling="spectral"), dict(graft="lion"),
+    dict(evd_heuristic="relu"), dict(root_p=3), dict(block_size=-1), dict(precond_every=0),
+    dict(stats_every=0), dict(iters=0), dict(eps=-1e-6), dict(eps=float("nan")),
+    dict(scaling="power", pi_vectors=12), dict(method="evd", block_size=256), dict(one_sided=(5,)),
+])
+def test_config_check_refuses_bad_options(bad):
+    cfg = OPT.ShampooConfig(**bad)
+    with pytest.raises(ValueError):
+        cfg.check(n_layers=3)
+
+
+def test_config_check_accepts_the_workload_settings():
+    OPT.ShampooConfig().check(3)
+    OPT.ShampooConfig(method="cheb", iters=0).check()
+    OPT.ShampooConfig(method="evd", block_size=128, evd_heuristic="shmp", one_sided=(0, 2)).check(3)
+    OPT.ShampooConfig(scaling="power", pi_vectors=16, dtype="tf32", graft="adam", root_p=8).check()

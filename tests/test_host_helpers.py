@@ -58,3 +58,40 @@ def test_config_check_accepts_the_workload_settings():
     OPT.ShampooConfig(method="cheb", iters=0).check()
     OPT.ShampooConfig(method="evd", block_size=128, evd_heuristic="shmp", one_sided=(0, 2)).check(3)
     OPT.ShampooConfig(scaling="power", pi_vectors=16, dtype="tf32", graft="adam", root_p=8).check()
+
+
+def test_bench_reference_arm_json_contract():
+    """bench.py --impl reference prints one JSON line with the keys the
+    driver reads (on the host cores, no GPU)."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config",
+                          "tiny_dense", "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=300, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] == 3 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+
+
+@pytest.mark.parametrize("config", ["spd_stack", "evd_stack"])
+def test_bench_reference_arm_for_root_only_workloads(config):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", config],
+                         capture_output=True, text=True, timeout=120, cwd=root)
+    assert out.returncode == 0
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
+    assert d["impl"] == "reference" and "unavailable" in d

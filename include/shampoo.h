@@ -25,7 +25,8 @@
  *   - Invalid arguments are reported before anything is enqueued; the call
  *     then returns a nonzero shp_status and shampoo_last_error() describes it.
  *     Numerical failure of an iteration is not an error: it is written to the
- *     per-matrix status array of shampoo_inv_root.
+ *     per-matrix status array of the root calls (shampoo_inv_root and its
+ *     _static, _warm and _evd forms).
  */
 #ifndef SHAMPOO_H
 #define SHAMPOO_H

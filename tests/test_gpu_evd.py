@@ -157,3 +157,24 @@ def test_evd_roots_in_the_step(heuristic):
         print(f"EVD {heuristic} step {t + 1}: W vs oracle {err:.2e}")
         assert err < 1e-3
     assert all(((s.cpu().numpy() & 0xff) == 0).all() for s in opt.status)
+
+
+def test_evd_nonfinite_is_per_matrix():
+    """A NaN in one matrix of the stack flags that matrix (SHP_ROOT_NONFINITE)
+    and leaves the others bit-identical to a clean run: one CTA per matrix,
+    no reduction across matrices, the sweep count bounded."""
+    import torch
+    rng = np.random.default_rng(46)
+    L = np.stack([g @ g.T for g in rng.standard_normal((4, 64, 96))]).astype(np.float32)
+    X0, _, st0 = B.inv_root_evd(to_dev(L), 1e-4, "corrected")
+    bad = L.copy()
+    bad[2, 3, 5] = np.nan
+    X1, _, st1 = B.inv_root_evd(to_dev(bad), 1e-4, "corrected")
+    torch.cuda.synchronize()
+    st0, st1 = st0.cpu().numpy(), st1.cpu().numpy()
+    assert ((st0 & 0xff) == 0).all()
+    assert st1[2] & 1
+    assert all((st1[b] & 0xff) == 0 for b in (0, 1, 3))
+    X0, X1 = X0.cpu().numpy(), X1.cpu().numpy()
+    for b in (0, 1, 3):
+        assert np.array_equal(X0[b], X1[b])

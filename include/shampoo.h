@@ -308,7 +308,8 @@ SHP_API shp_status shampoo_inv_root_warm(const float* A, const float* X0, int32_
  * matrix's status gets SHP_ROOT_UNCONVERGED).
  * A: device (count, n, n) float32 row-major; X_out: same shape (may be A);
  * eig_out: NULL or device (count, n) float32, lambda ascending per matrix;
- * status_out: device [count] int32, SHP_ROOT_* bits in bits 0-7 and the
+ * status_out: device [count] int32, SHP_ROOT_* bits in bits 0-7
+ *   (SHP_ROOT_NONFINITE also when A itself holds a NaN / Inf) and the
  *   number of sweeps taken in bits 8-15 (the final sweep, which rotates
  *   nothing, included).
  * Sizes: 1 <= n <= SHP_EVD_MAX_N (any n), count >= 1; p in {2, 4, 8}.

@@ -72,9 +72,12 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
   const long long nn = (long long)n * n;
   const float* Ab = A + (long long)blockIdx.x * nn;
 
+  bool bad_in = false;  // a NaN / Inf in A: the rotation test skips such entries, so flag it here
   for (int i = tid; i < n * n; i += blockDim.x) {
     const int r = i / n, c = i - r * n;
-    a[r * ld + c] = (double)Ab[i];
+    const float x = Ab[i];
+    bad_in |= !isfinite(x);
+    a[r * ld + c] = (double)x;
     v[r * ld + c] = r == c ? 1.f : 0.f;
   }
   if (tid == 0) {
@@ -82,6 +85,7 @@ __global__ void __launch_bounds__(kEvdThreads, 1)
     flags = 0;
   }
   __syncthreads();
+  if (bad_in) atomicOr(&flags, SHP_ROOT_NONFINITE);
   for (int i = tid; i < n * n; i += blockDim.x) {  // symmetrise, damp
     const int r = i / n, c = i - r * n;
     if (r < c) {

@@ -144,6 +144,32 @@ class BlockedShampoo:
         self._graphs = {}       # (fresh roots?, gradient addresses) -> (CUDAGraph, library launches in it)
         self.graph_launches = 0  # library kernel launches replayed from graphs so far
 
+    def state_dict(self) -> dict:
+        """The optimizer state as host tensors -- step count, statistics,
+        the current roots (reused until the next refresh), graft moments --
+        so that a run can be checkpointed and resumed; the weights stay with
+        the caller."""
+        def host(ts):
+            return None if ts is None else [t.detach().to("cpu", copy=True) for t in ts]
+        return {"t": self.t, "shapes": [list(s) for s in self.shapes], "factors": host(self.factors),
+                "roots": host(self.roots), "m": host(self.m), "v": host(self.v)}
+
+    def load_state_dict(self, state: dict) -> None:
+        """Restores ``state_dict()`` output of an optimizer with the same
+        shapes and configuration (copied into the existing device tensors, so
+        captured CUDA graphs stay valid)."""
+        if [tuple(int(x) for x in s) for s in state["shapes"]] != self.shapes:
+            raise ValueError("state was saved for other layer shapes")
+        for name in ("factors", "roots", "m", "v"):
+            dst, src = getattr(self, name), state[name]
+            if (dst is None) != (src is None) or (dst is not None and len(dst) != len(src)):
+                raise ValueError(f"state entry {name!r} does not match this optimizer's configuration")
+            for d, x in zip(dst or [], src or []):
+                if tuple(d.shape) != tuple(x.shape):
+                    raise ValueError(f"state entry {name!r} has shape {tuple(x.shape)}, expected {tuple(d.shape)}")
+                d.copy_(x)
+        self.t = int(state["t"])
+
     def _direction(self, G, stream, fresh: bool, stats: bool = True) -> None:
         """Stack, statistics (when ``stats``), roots (when fresh) and D for
         gradients G."""
